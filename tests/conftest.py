@@ -1,0 +1,21 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line(
+        "markers", "gpu: needs a B200 (sm_100a); fails rather than skips when no GPU is present")
+
+
+@pytest.fixture(scope="session")
+def cuda_device():
+    """The CUDA device for GPU tests.  A missing GPU is a failure, not a skip."""
+    import torch
+    assert torch.cuda.is_available(), "GPU test selected but no CUDA device is visible"
+    return torch.device("cuda", 0)
