@@ -1,0 +1,190 @@
+"""Python binding of libnvfp4, the NVFP4 linear layer for B200 (sm_100a).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  The functions carry the names of the C entry points declared in
+``include/nvfp4.h`` and take torch CUDA tensors for device memory; outputs and
+workspaces not passed in are allocated with torch (the library itself never
+allocates).  Every call is enqueued on the current torch stream.
+
+There is no fallback: if ``libnvfp4.so`` has not been built, importing the
+library raises ``ImportError``; a non-zero status raises :class:`NVFP4Error`.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
+
+# status codes, enumerations (values of include/nvfp4.h)
+OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_DTYPE, ERR_WORKSPACE, ERR_ARCH, ERR_LAUNCH, ERR_LAYOUT, ERR_MODE, \
+    ERR_DEVICE_TIMEOUT = range(11)
+DTYPE_F32, DTYPE_BF16 = 0, 1
+SF_ROWMAJOR, SF_TILED = 0, 1
+MODE_AUTO, MODE_W4A16, MODE_W4A4 = 0, 1, 2
+EPI_NONE, EPI_SWIGLU, EPI_COMBINE = 0, 1, 2
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status: int, call: str):
+        super().__init__(f"{call} failed: {status_string(status)} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libnvfp4 (raises ImportError when it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m bit_linear_moe_b200.build` "
+                              "(there is no fallback implementation)")
+        L = ctypes.CDLL(LIB_PATH)
+        p, i64, i32, sz, i = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t, ctypes.c_int
+        sig = {
+            "nvfp4_status_string": (ctypes.c_char_p, [i]),
+            "nvfp4_version": (i, []),
+            "nvfp4_scales_bytes": (sz, [i64, i64, i]),
+            "nvfp4_read_device_status": (i, [p, p]),
+            "nvfp4_quantize_workspace": (sz, [i64, i64]),
+            "nvfp4_quantize": (i, [p, i, i64, i64, p, i, p, p, p, p, sz, p]),
+            "nvfp4_linear_workspace": (sz, [i64, i64, i64, i]),
+            "nvfp4_linear": (i, [p, i, i64, i64, p, p, i, p, i64, p, i, i, p, sz, p]),
+            "moe_route_topk_workspace": (sz, [i64, i32, i32]),
+            "moe_route_topk": (i, [p, p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p, sz, p]),
+            "moe_grouped_linear_workspace": (sz, [i64, i64, i64, i32, i32, i, i]),
+            "moe_grouped_linear": (i, [p, i, i64, i, p, p, i32, i64, p, p, i, p, i64, i, p, p, i32, p, i, i,
+                                       p, sz, p]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().nvfp4_status_string(int(status)).decode()
+
+
+def _check(status: int, call: str):
+    if status != OK:
+        raise NVFP4Error(status, call)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _workspace(nbytes: int, device, ws=None):
+    if nbytes == 0:
+        return None, 0
+    if ws is None:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return ws, ws.numel() * ws.element_size()
+
+
+def nvfp4_scales_bytes(rows: int, cols: int, sf_layout: int) -> int:
+    return int(lib().nvfp4_scales_bytes(rows, cols, sf_layout))
+
+
+def nvfp4_quantize(x: torch.Tensor, gs_in: torch.Tensor | None = None, sf_layout: int = SF_ROWMAJOR,
+                   codes=None, scales=None, gs_out=None, ws=None):
+    """Quantize ``x [rows, cols]`` (fp32 or bf16) to ``(codes, scales, gs)`` on the device."""
+    rows, cols = x.shape
+    dev = x.device
+    if codes is None:
+        codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(nvfp4_scales_bytes(rows, cols, sf_layout), dtype=torch.uint8, device=dev)
+    if gs_out is None:
+        gs_out = torch.empty(1, dtype=torch.float32, device=dev)
+    ws, wsb = _workspace(int(lib().nvfp4_quantize_workspace(rows, cols)), dev, ws)
+    _check(lib().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, _ptr(gs_in), sf_layout, _ptr(codes),
+                                _ptr(scales), _ptr(gs_out), _ptr(ws), wsb, _stream()), "nvfp4_quantize")
+    return codes, scales, gs_out
+
+
+def nvfp4_linear(x: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, w_gs: torch.Tensor,
+                 w_sf_layout: int = SF_ROWMAJOR, y=None, y_dtype=torch.float32, mode: int = MODE_AUTO, ws=None):
+    """``y = x @ W^T`` with W NVFP4 ``(w_codes [N, K/2], w_scales, w_gs)``; x bf16 [M, K]."""
+    M, K = x.shape
+    N = w_codes.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=x.device)
+    ws, wsb = _workspace(int(lib().nvfp4_linear_workspace(M, K, N, mode)), x.device, ws)
+    _check(lib().nvfp4_linear(_ptr(x), _dtype_code(x), M, K, _ptr(w_codes), _ptr(w_scales), w_sf_layout,
+                              _ptr(w_gs), N, _ptr(y), _dtype_code(y), mode, _ptr(ws), wsb, _stream()),
+           "nvfp4_linear")
+    return y
+
+
+def moe_route_topk(h: torch.Tensor, w_router: torch.Tensor, k: int, logit_bias=None, want_logits: bool = False,
+                   out=None, ws=None):
+    """Router, top-k and permutation.  Returns a dict of device tensors:
+    ``logits`` (if wanted), ``topk_idx``, ``topk_w``, ``expert_offsets``, ``perm_tok``, ``perm_slot``, ``row_of``."""
+    T, H = h.shape
+    E = w_router.shape[0]
+    dev = h.device
+    o = dict(out or {})
+    if want_logits and "logits" not in o:
+        o["logits"] = torch.empty((T, E), dtype=torch.float32, device=dev)
+    o.setdefault("topk_idx", torch.empty((T, k), dtype=torch.int32, device=dev))
+    o.setdefault("topk_w", torch.empty((T, k), dtype=torch.float32, device=dev))
+    o.setdefault("expert_offsets", torch.empty(E + 1, dtype=torch.int32, device=dev))
+    o.setdefault("perm_tok", torch.empty(T * k, dtype=torch.int32, device=dev))
+    o.setdefault("perm_slot", torch.empty(T * k, dtype=torch.int32, device=dev))
+    o.setdefault("row_of", torch.empty((T, k), dtype=torch.int32, device=dev))
+    ws, wsb = _workspace(int(lib().moe_route_topk_workspace(T, E, k)), dev, ws)
+    _check(lib().moe_route_topk(_ptr(h), _ptr(w_router), _ptr(logit_bias), T, H, E, k, _ptr(o.get("logits")),
+                                _ptr(o["topk_idx"]), _ptr(o["topk_w"]), _ptr(o["expert_offsets"]),
+                                _ptr(o["perm_tok"]), _ptr(o["perm_slot"]), _ptr(o["row_of"]), _ptr(ws), wsb,
+                                _stream()), "moe_route_topk")
+    return o
+
+
+def moe_grouped_linear(x: torch.Tensor, expert_offsets: torch.Tensor, w_codes: torch.Tensor,
+                       w_scales: torch.Tensor, w_gs: torch.Tensor, R: int, perm_tok=None, gather: bool = True,
+                       w_sf_layout: int = SF_ROWMAJOR, epilogue: int = EPI_NONE, topk_w=None, row_of=None,
+                       k: int = 0, y=None, y_dtype=torch.float32, mode: int = MODE_AUTO, ws=None):
+    """Expert linears over permuted rows; see ``moe_grouped_linear`` in ``include/nvfp4.h``."""
+    K = x.shape[1]
+    E, N = w_codes.shape[0], w_codes.shape[1]
+    if y is None:
+        if epilogue == EPI_SWIGLU:
+            shape = (R, N // 2)
+        elif epilogue == EPI_COMBINE:
+            shape = (R // k, N)
+        else:
+            shape = (R, N)
+        y = torch.empty(shape, dtype=y_dtype, device=x.device)
+    ws, wsb = _workspace(int(lib().moe_grouped_linear_workspace(R, K, N, E, k, epilogue, mode)), x.device, ws)
+    _check(lib().moe_grouped_linear(_ptr(x), _dtype_code(x), K, int(gather), _ptr(expert_offsets),
+                                    _ptr(perm_tok), E, R, _ptr(w_codes), _ptr(w_scales), w_sf_layout, _ptr(w_gs),
+                                    N, epilogue, _ptr(topk_w), _ptr(row_of), k, _ptr(y), _dtype_code(y), mode,
+                                    _ptr(ws), wsb, _stream()), "moe_grouped_linear")
+    return y
+
+
+def nvfp4_read_device_status() -> int:
+    st = ctypes.c_int(0)
+    _check(lib().nvfp4_read_device_status(_stream(), ctypes.byref(st)), "nvfp4_read_device_status")
+    return st.value

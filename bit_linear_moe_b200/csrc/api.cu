@@ -1,0 +1,289 @@
+// libnvfp4 C ABI: argument validation, workspace layout and dispatch.
+// The declarations, argument meanings, layouts and error behaviour are in
+// include/nvfp4.h.  Every entry point validates on the host and returns an
+// error before launching anything.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4 {
+__device__ int g_device_status = 0;
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+static size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+// The current device must be sm_100 (B200 / GB200 class).  Cached per device.
+static int check_arch() {
+    static int cache[64] = {0};  // 0 unknown, 1 ok, 2 bad
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_ARCH;
+    if (dev < 0 || dev >= 64) return NVFP4_ERR_ARCH;
+    if (cache[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return NVFP4_ERR_ARCH;
+        cache[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    }
+    return cache[dev] == 1 ? NVFP4_OK : NVFP4_ERR_ARCH;
+}
+
+static bool dtype_ok(int d) { return d == NVFP4_DTYPE_F32 || d == NVFP4_DTYPE_BF16; }
+static bool layout_ok(int l) { return l == NVFP4_SF_ROWMAJOR || l == NVFP4_SF_TILED; }
+
+static size_t scales_bytes(int64_t rows, int64_t cols, int layout) {
+    if (rows < 1 || cols < 16 || cols % 16) return 0;
+    const int64_t nsf = cols / 16;
+    if (layout == NVFP4_SF_ROWMAJOR) return (size_t)(rows * nsf);
+    if (layout == NVFP4_SF_TILED) return (size_t)((rows + 127) / 128 * 128) * (size_t)((nsf + 3) / 4 * 4);
+    return 0;
+}
+
+// Row padding of a W4A4 operand: the tensor-core tiles are 128 rows.
+static int64_t moe_w4a4_rows(int64_t R, int32_t E) { return R + (int64_t)E * 127; }
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+#define NVFP4_TRY(expr)                 \
+    do {                                \
+        const int _s = (expr);          \
+        if (_s != NVFP4_OK) return _s;  \
+    } while (0)
+
+extern "C" {
+
+const char* nvfp4_status_string(int status) {
+    switch (status) {
+        case NVFP4_OK: return "ok";
+        case NVFP4_ERR_NULL: return "a required pointer is NULL";
+        case NVFP4_ERR_SHAPE: return "a size is out of range or not a required multiple";
+        case NVFP4_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case NVFP4_ERR_DTYPE: return "unsupported dtype";
+        case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+        case NVFP4_ERR_ARCH: return "the current device is not sm_100";
+        case NVFP4_ERR_LAUNCH: return "a kernel launch or driver call failed";
+        case NVFP4_ERR_LAYOUT: return "scale layout not accepted by this mode";
+        case NVFP4_ERR_MODE: return "unknown mode or epilogue";
+        case NVFP4_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out";
+        default: return "unknown status";
+    }
+}
+
+int nvfp4_version(void) { return 100; }
+
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int sf_layout) { return scales_bytes(rows, cols, sf_layout); }
+
+int nvfp4_read_device_status(void* stream, int* status_out) {
+    if (!status_out) return NVFP4_ERR_NULL;
+    cudaStream_t st = (cudaStream_t)stream;
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(int), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return NVFP4_ERR_LAUNCH;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return NVFP4_ERR_LAUNCH;
+    if (cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return NVFP4_ERR_LAUNCH;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return NVFP4_ERR_LAUNCH;
+    *status_out = v;
+    return NVFP4_OK;
+}
+
+// ---- quantize ----------------------------------------------------------------
+
+size_t nvfp4_quantize_workspace(int64_t rows, int64_t cols) {
+    (void)rows;
+    (void)cols;
+    return 256;
+}
+
+int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t cols, const float* gs_in, int sf_layout,
+                   uint8_t* codes, uint8_t* scales, float* gs_out, void* ws, size_t ws_bytes, void* stream) {
+    if (!x || !codes || !scales || !gs_out) return NVFP4_ERR_NULL;
+    if (!dtype_ok(x_dtype)) return NVFP4_ERR_DTYPE;
+    if (!layout_ok(sf_layout)) return NVFP4_ERR_LAYOUT;
+    if (rows < 1 || cols < 16 || cols % 16 || rows > (int64_t)1 << 31 || cols > (int64_t)1 << 31)
+        return NVFP4_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales)) return NVFP4_ERR_ALIGN;
+    if (!ws || ws_bytes < nvfp4_quantize_workspace(rows, cols)) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NVFP4_ERR_ALIGN;
+    NVFP4_TRY(check_arch());
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned* amax = (unsigned*)ws;
+    if (!gs_in) NVFP4_TRY(launch_amax(x, x_dtype, rows * cols, amax, st));
+    return launch_quantize(x, x_dtype, nullptr, rows, cols, sf_layout, gs_in, amax, codes, scales, gs_out, st);
+}
+
+// ---- linear --------------------------------------------------------------------
+
+static int resolve_mode(int mode, int64_t M) {
+    if (mode == NVFP4_MODE_AUTO) return M <= 32 ? NVFP4_MODE_W4A16 : NVFP4_MODE_W4A4;
+    return mode;
+}
+
+size_t nvfp4_linear_workspace(int64_t M, int64_t K, int64_t N, int mode) {
+    (void)N;
+    mode = resolve_mode(mode, M);
+    if (mode == NVFP4_MODE_W4A4) {
+        // amax word, gs, activation codes, tiled activation scales
+        return align256(256) + align256((size_t)(M * K / 2)) + align256(scales_bytes(M, K, NVFP4_SF_TILED));
+    }
+    return 0;
+}
+
+int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t* w_codes, const uint8_t* w_scales,
+                 int w_sf_layout, const float* w_gs, int64_t N, void* y, int y_dtype, int mode, void* ws,
+                 size_t ws_bytes, void* stream) {
+    if (!x || !w_codes || !w_scales || !w_gs || !y) return NVFP4_ERR_NULL;
+    if (x_dtype != NVFP4_DTYPE_BF16 || !dtype_ok(y_dtype)) return NVFP4_ERR_DTYPE;
+    if (!layout_ok(w_sf_layout)) return NVFP4_ERR_LAYOUT;
+    if (mode != NVFP4_MODE_AUTO && mode != NVFP4_MODE_W4A16 && mode != NVFP4_MODE_W4A4) return NVFP4_ERR_MODE;
+    if (M < 1 || N < 1 || K < 16 || K % 16 || M > ((int64_t)1 << 31) || N > ((int64_t)1 << 31) ||
+        K > ((int64_t)1 << 24))
+        return NVFP4_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y)) return NVFP4_ERR_ALIGN;
+    mode = resolve_mode(mode, M);
+    if (mode == NVFP4_MODE_W4A4) {
+        if (w_sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_LAYOUT;
+        if (K % 256) return NVFP4_ERR_SHAPE;
+    }
+    const size_t need = nvfp4_linear_workspace(M, K, N, mode);
+    if (need && (!ws || ws_bytes < need)) return NVFP4_ERR_WORKSPACE;
+    if (need && !aligned16(ws)) return NVFP4_ERR_ALIGN;
+    NVFP4_TRY(check_arch());
+    if (mode == NVFP4_MODE_W4A4) return NVFP4_ERR_MODE;  // tensor-core path not wired yet
+    GemvArgs a{};
+    a.x = x;
+    a.M = M;
+    a.K = K;
+    a.codes = w_codes;
+    a.scales = w_scales;
+    a.sf_layout = w_sf_layout;
+    a.gs = w_gs;
+    a.N = N;
+    a.E = 1;
+    a.epilogue = NVFP4_EPI_NONE;
+    a.y = y;
+    a.y_dtype = y_dtype;
+    a.ldy = N;
+    return launch_gemv_w4a16(a, (cudaStream_t)stream);
+}
+
+// ---- MoE routing -------------------------------------------------------------------
+
+static int64_t perm_blocks(int64_t T) { return (T + kPermBlockTokens - 1) / kPermBlockTokens; }
+
+size_t moe_route_topk_workspace(int64_t T, int32_t E, int32_t k) {
+    (void)k;
+    if (T < 1 || E < 1) return 0;
+    return align256((size_t)(T * E) * 4) + 2 * align256((size_t)(perm_blocks(T) * E) * 4);
+}
+
+int moe_route_topk(const void* h, const void* w_router, const float* logit_bias, int64_t T, int64_t H, int32_t E,
+                   int32_t k, float* logits_out, int32_t* topk_idx, float* topk_w, int32_t* expert_offsets,
+                   int32_t* perm_tok, int32_t* perm_slot, int32_t* row_of, void* ws, size_t ws_bytes,
+                   void* stream) {
+    if (!h || !w_router || !topk_idx || !topk_w || !expert_offsets || !perm_tok || !perm_slot || !row_of)
+        return NVFP4_ERR_NULL;
+    if (T < 1 || T > ((int64_t)1 << 24) || H < 8 || H % 8 || E < 1 || E > 1024 || k < 1 || k > 32 || k > E)
+        return NVFP4_ERR_SHAPE;
+    if (!aligned16(h) || !aligned16(w_router)) return NVFP4_ERR_ALIGN;
+    if (!ws || ws_bytes < moe_route_topk_workspace(T, E, k)) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NVFP4_ERR_ALIGN;
+    NVFP4_TRY(check_arch());
+    cudaStream_t st = (cudaStream_t)stream;
+    char* p = (char*)ws;
+    float* logits = (float*)p;
+    p += align256((size_t)(T * E) * 4);
+    int32_t* blk_counts = (int32_t*)p;
+    p += align256((size_t)(perm_blocks(T) * E) * 4);
+    int32_t* blk_base = (int32_t*)p;
+    if (logits_out) logits = logits_out;
+    NVFP4_TRY(launch_router_logits(h, w_router, logit_bias, T, H, E, logits, st));
+    NVFP4_TRY(launch_topk_count(logits, T, E, k, topk_idx, topk_w, blk_counts, st));
+    NVFP4_TRY(launch_perm_scan(blk_counts, perm_blocks(T), E, expert_offsets, blk_base, st));
+    return launch_perm_scatter(topk_idx, T, E, k, blk_base, perm_tok, perm_slot, row_of, st);
+}
+
+// ---- MoE grouped linear ------------------------------------------------------------
+
+static int resolve_grouped_mode(int mode, int64_t R) {
+    if (mode == NVFP4_MODE_AUTO) return R <= 512 ? NVFP4_MODE_W4A16 : NVFP4_MODE_W4A4;
+    return mode;
+}
+
+size_t moe_grouped_linear_workspace(int64_t R, int64_t K, int64_t N, int32_t E, int32_t k, int epilogue, int mode) {
+    (void)k;
+    mode = resolve_grouped_mode(mode, R);
+    size_t need = 0;
+    if (epilogue == NVFP4_EPI_COMBINE) need += align256((size_t)(R * N) * 4);
+    if (mode == NVFP4_MODE_W4A4) {
+        const int64_t rp = moe_w4a4_rows(R, E);
+        need += align256(256) + align256((size_t)(rp * K / 2)) + align256(scales_bytes(rp, K, NVFP4_SF_TILED)) +
+                align256((size_t)rp * 4);
+    }
+    return need;
+}
+
+int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const int32_t* expert_offsets,
+                       const int32_t* perm_tok, int32_t E, int64_t R, const uint8_t* w_codes,
+                       const uint8_t* w_scales, int w_sf_layout, const float* w_gs, int64_t N, int epilogue,
+                       const float* topk_w, const int32_t* row_of, int32_t k, void* y, int y_dtype, int mode,
+                       void* ws, size_t ws_bytes, void* stream) {
+    if (!x || !expert_offsets || !w_codes || !w_scales || !w_gs || !y) return NVFP4_ERR_NULL;
+    if (gather && !perm_tok) return NVFP4_ERR_NULL;
+    if (x_dtype != NVFP4_DTYPE_BF16 || !dtype_ok(y_dtype)) return NVFP4_ERR_DTYPE;
+    if (!layout_ok(w_sf_layout)) return NVFP4_ERR_LAYOUT;
+    if (epilogue != NVFP4_EPI_NONE && epilogue != NVFP4_EPI_SWIGLU && epilogue != NVFP4_EPI_COMBINE)
+        return NVFP4_ERR_MODE;
+    if (mode != NVFP4_MODE_AUTO && mode != NVFP4_MODE_W4A16 && mode != NVFP4_MODE_W4A4) return NVFP4_ERR_MODE;
+    if (E < 1 || E > 1024 || R < 1 || R > ((int64_t)1 << 26) || N < 1 || N > ((int64_t)1 << 20) || K < 16 ||
+        K % 16 || K > ((int64_t)1 << 20))
+        return NVFP4_ERR_SHAPE;
+    if (epilogue == NVFP4_EPI_SWIGLU && N % 2) return NVFP4_ERR_SHAPE;
+    if (epilogue == NVFP4_EPI_COMBINE) {
+        if (!topk_w || !row_of) return NVFP4_ERR_NULL;
+        if (k < 1 || R % k || N % 4) return NVFP4_ERR_SHAPE;
+    }
+    if (!aligned16(x) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y)) return NVFP4_ERR_ALIGN;
+    mode = resolve_grouped_mode(mode, R);
+    if (mode == NVFP4_MODE_W4A4) {
+        if (w_sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_LAYOUT;
+        if (K % 256) return NVFP4_ERR_SHAPE;
+    }
+    const size_t need = moe_grouped_linear_workspace(R, K, N, E, k, epilogue, mode);
+    if (need && (!ws || ws_bytes < need)) return NVFP4_ERR_WORKSPACE;
+    if (need && !aligned16(ws)) return NVFP4_ERR_ALIGN;
+    NVFP4_TRY(check_arch());
+    if (mode == NVFP4_MODE_W4A4) return NVFP4_ERR_MODE;  // tensor-core path not wired yet
+    cudaStream_t st = (cudaStream_t)stream;
+    GemvArgs a{};
+    a.x = x;
+    a.gather = gather ? perm_tok : nullptr;
+    a.M = R;
+    a.K = K;
+    a.codes = w_codes;
+    a.scales = w_scales;
+    a.sf_stride = (int64_t)scales_bytes(N, K, w_sf_layout);
+    a.sf_layout = w_sf_layout;
+    a.gs = w_gs;
+    a.N = N;
+    a.offsets = expert_offsets;
+    a.E = E;
+    if (epilogue == NVFP4_EPI_COMBINE) {
+        float* d = (float*)ws;
+        a.epilogue = NVFP4_EPI_NONE;
+        a.y = d;
+        a.y_dtype = NVFP4_DTYPE_F32;
+        a.ldy = N;
+        NVFP4_TRY(launch_gemv_w4a16(a, st));
+        return launch_combine(d, topk_w, row_of, R / k, k, N, y, y_dtype, st);
+    }
+    a.epilogue = epilogue;
+    a.y = y;
+    a.y_dtype = y_dtype;
+    a.ldy = epilogue == NVFP4_EPI_SWIGLU ? N / 2 : N;
+    return launch_gemv_w4a16(a, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,51 @@
+// Internal launchers behind the C ABI (not exported).  Every launcher takes
+// validated arguments and returns an NVFP4_* status.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nvfp4 {
+
+// quantize.cu
+int launch_amax(const void* x, int x_dtype, int64_t n, unsigned* amax_bits, cudaStream_t st);
+int launch_quantize(const void* x, int x_dtype, const int32_t* src_rows, int64_t dst_rows, int64_t cols,
+                    int sf_layout, const float* gs_in, const unsigned* amax_bits, uint8_t* codes,
+                    uint8_t* scales, float* gs_out, cudaStream_t st);
+
+// gemv.cu: W4A16 on CUDA cores.
+struct GemvArgs {
+    const void* x;            // bf16 activations, row stride K
+    const int32_t* gather;    // grouped: activation row of output row r is gather[r] (nullable)
+    int64_t M;                // dense: number of rows of x / y
+    int64_t K;
+    const uint8_t* codes;     // [N, K/2]  (grouped: [E, N, K/2])
+    const uint8_t* scales;    // per-matrix scale block (grouped: E of them, sf_stride apart)
+    int64_t sf_stride;        // bytes between experts' scale blocks
+    int sf_layout;
+    const float* gs;          // [1] or [E]
+    int64_t N;                // weight rows
+    const int32_t* offsets;   // grouped: [E+1] row offsets (nullable for dense)
+    int32_t E;
+    int epilogue;             // NVFP4_EPI_NONE or NVFP4_EPI_SWIGLU
+    void* y;                  // output rows
+    int y_dtype;              // NVFP4_DTYPE_F32 / BF16
+    int64_t ldy;              // elements per output row
+};
+int launch_gemv_w4a16(const GemvArgs& a, cudaStream_t st);
+
+// moe.cu
+int launch_router_logits(const void* h, const void* wr, const float* bias, int64_t T, int64_t H, int32_t E,
+                         float* logits, cudaStream_t st);
+int launch_topk_count(const float* logits, int64_t T, int32_t E, int32_t k, int32_t* topk_idx, float* topk_w,
+                      int32_t* blk_counts, cudaStream_t st);
+int launch_perm_scan(const int32_t* blk_counts, int64_t nblk, int32_t E, int32_t* offsets, int32_t* blk_base,
+                     cudaStream_t st);
+int launch_perm_scatter(const int32_t* topk_idx, int64_t T, int32_t E, int32_t k, const int32_t* blk_base,
+                        int32_t* perm_tok, int32_t* perm_slot, int32_t* row_of, cudaStream_t st);
+int launch_combine(const float* d, const float* topk_w, const int32_t* row_of, int64_t T, int32_t k, int64_t N,
+                   void* y, int y_dtype, cudaStream_t st);
+
+constexpr int kPermBlockTokens = 128;
+
+}  // namespace nvfp4

@@ -1,0 +1,265 @@
+// K5/K6/K8: router, top-k, token permutation and combine of a routed
+// mixture-of-experts layer (CHImp Alpha v1.0 model card, "How it fits on one
+// GPU": each token is routed to 10 of 512 experts per layer).
+//
+// Router logits  l[t, e] = sum_h h[t, h] * Wr[e, h] (+ bias[e]), bf16 inputs,
+//                fp32 accumulation (products of two bf16 are exact in fp32;
+//                sums are kept in 32-term tile partials).
+// Top-k          one warp per token; k rounds of a warp arg-max that orders by
+//                (logit descending, expert index ascending); weights are the
+//                softmax over the k winners.
+// Permutation    counting sort by expert, stable in token order, without
+//                atomics on the result: per block of 128 tokens a bitmask per
+//                expert marks the tokens that chose it, so a token's rank inside
+//                its block is a popcount; block bases come from a scan.
+// Combine        y[t, n] = sum_j w[t, j] * d[row_of[t, j], n], j ascending.
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4 {
+
+// ---- router logits: 64 x 64 output tile per CTA, 256 threads, 4 x 4 each ----
+constexpr int RT = 64, RK = 32;
+
+__global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16* __restrict__ h,
+                                                            const __nv_bfloat16* __restrict__ wr,
+                                                            const float* __restrict__ bias, int64_t T,
+                                                            int64_t H, int32_t E, float* __restrict__ logits) {
+    __shared__ float sh[RK][RT + 1];
+    __shared__ float sw[RK][RT + 1];
+    const int tid = threadIdx.x;
+    const int64_t t0 = (int64_t)blockIdx.x * RT, e0 = (int64_t)blockIdx.y * RT;
+    const int ty = tid / 16, tx = tid % 16;  // 16 x 16 threads, 4 x 4 outputs each
+    float acc[4][4] = {};
+    for (int64_t k0 = 0; k0 < H; k0 += RK) {
+        // load 64 rows x 32 cols of h and of wr (bf16 -> fp32), 8 elements per thread
+        {
+            const int r = tid / 4, q = (tid % 4) * 8;
+            float hv[8] = {}, wv[8] = {};
+            if (t0 + r < T && k0 + q < H) {
+                uint4 v = ldg_v4(h + (t0 + r) * H + k0 + q);
+                uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) { hv[2 * j] = bf16lo_to_f32(u[j]); hv[2 * j + 1] = bf16hi_to_f32(u[j]); }
+            }
+            if (e0 + r < E && k0 + q < H) {
+                uint4 v = ldg_v4(wr + (e0 + r) * H + k0 + q);
+                uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) { wv[2 * j] = bf16lo_to_f32(u[j]); wv[2 * j + 1] = bf16hi_to_f32(u[j]); }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { sh[q + j][r] = hv[j]; sw[q + j][r] = wv[j]; }
+        }
+        __syncthreads();
+        float part[4][4] = {};
+#pragma unroll 8
+        for (int kk = 0; kk < RK; ++kk) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { a[i] = sh[kk][ty * 4 + i]; b[i] = sw[kk][tx * 4 + i]; }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) part[i][j] = fmaf(a[i], b[j], part[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int64_t t = t0 + ty * 4 + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t e = e0 + tx * 4 + j;
+            if (e < E) logits[t * E + e] = acc[i][j] + (bias ? bias[e] : 0.0f);
+        }
+    }
+}
+
+int launch_router_logits(const void* h, const void* wr, const float* bias, int64_t T, int64_t H, int32_t E,
+                         float* logits, cudaStream_t st) {
+    dim3 grid((unsigned)((T + RT - 1) / RT), (unsigned)((E + RT - 1) / RT));
+    router_logits_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)h, (const __nv_bfloat16*)wr, bias, T, H, E,
+                                               logits);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+}
+
+// ---- top-k + per-block expert counts ------------------------------------
+// CTA = 256 threads = 8 warps, kPermBlockTokens tokens; a warp takes 16 tokens.
+constexpr int kMaxE = 1024, kMaxPerLane = kMaxE / 32;
+
+NVFP4_DEV bool better(float v, int i, float bv, int bi) { return v > bv || (v == bv && i < bi); }
+
+__global__ void __launch_bounds__(256) topk_count_kernel(const float* __restrict__ logits, int64_t T, int32_t E,
+                                                         int32_t k, int32_t* __restrict__ topk_idx,
+                                                         float* __restrict__ topk_w,
+                                                         int32_t* __restrict__ blk_counts) {
+    __shared__ uint32_t mask[kMaxE][kPermBlockTokens / 32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < E * (kPermBlockTokens / 32); i += blockDim.x) (&mask[0][0])[i] = 0;
+    __syncthreads();
+    const int64_t tb = (int64_t)blockIdx.x * kPermBlockTokens;
+    const int per_lane = (E + 31) / 32;
+    for (int tt = warp; tt < kPermBlockTokens; tt += 8) {
+        const int64_t t = tb + tt;
+        if (t >= T) break;
+        float v[kMaxPerLane];
+#pragma unroll
+        for (int i = 0; i < kMaxPerLane; ++i) {
+            const int e = i * 32 + lane;
+            v[i] = (i < per_lane && e < E) ? logits[t * E + e] : -INFINITY;
+        }
+        uint32_t taken = 0;  // bit i: v[i] already selected
+        float lmax = 0.0f, mywl = 0.0f;
+        int myidx = 0;
+        for (int j = 0; j < k; ++j) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < kMaxPerLane; ++i) {
+                const int e = i * 32 + lane;
+                if (i < per_lane && e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bi)) { bv = v[i]; bi = e; }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+            }
+            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+            if (j == 0) lmax = bv;
+            if (lane == j) { myidx = bi; mywl = bv; }
+        }
+        const float ex = lane < k ? expf(mywl - lmax) : 0.0f;
+        const float den = warp_sum(ex);
+        if (lane < k) {
+            topk_idx[t * k + lane] = myidx;
+            topk_w[t * k + lane] = ex / den;
+            atomicOr(&mask[myidx][tt >> 5], 1u << (tt & 31));
+        }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int c = 0;
+#pragma unroll
+        for (int w = 0; w < kPermBlockTokens / 32; ++w) c += __popc(mask[e][w]);
+        blk_counts[(int64_t)blockIdx.x * E + e] = c;
+    }
+}
+
+int launch_topk_count(const float* logits, int64_t T, int32_t E, int32_t k, int32_t* topk_idx, float* topk_w,
+                      int32_t* blk_counts, cudaStream_t st) {
+    const int64_t nblk = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+    topk_count_kernel<<<(unsigned)nblk, 256, 0, st>>>(logits, T, E, k, topk_idx, topk_w, blk_counts);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+}
+
+// ---- scan: expert offsets and per-block bases -----------------------------
+__global__ void __launch_bounds__(1024) perm_scan_kernel(const int32_t* __restrict__ blk_counts, int64_t nblk,
+                                                         int32_t E, int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ blk_base) {
+    __shared__ int32_t tot[kMaxE];
+    const int e = threadIdx.x;
+    int32_t run = 0;
+    if (e < E) {
+        for (int64_t b = 0; b < nblk; ++b) {
+            blk_base[b * E + e] = run;
+            run += blk_counts[b * E + e];
+        }
+    }
+    tot[e] = e < E ? run : 0;
+    __syncthreads();
+    // Hillis-Steele inclusive scan over 1024 entries.
+    for (int o = 1; o < kMaxE; o <<= 1) {
+        const int32_t add = e >= o ? tot[e - o] : 0;
+        __syncthreads();
+        tot[e] += add;
+        __syncthreads();
+    }
+    if (e < E) {
+        const int32_t excl = tot[e] - run;
+        offsets[e] = excl;
+        if (e == E - 1) offsets[E] = tot[e];
+        for (int64_t b = 0; b < nblk; ++b) blk_base[b * E + e] += excl;
+    }
+}
+
+int launch_perm_scan(const int32_t* blk_counts, int64_t nblk, int32_t E, int32_t* offsets, int32_t* blk_base,
+                     cudaStream_t st) {
+    perm_scan_kernel<<<1, kMaxE, 0, st>>>(blk_counts, nblk, E, offsets, blk_base);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+}
+
+// ---- scatter: one thread per token -----------------------------------------
+__global__ void __launch_bounds__(kPermBlockTokens) perm_scatter_kernel(
+    const int32_t* __restrict__ topk_idx, int64_t T, int32_t E, int32_t k, const int32_t* __restrict__ blk_base,
+    int32_t* __restrict__ perm_tok, int32_t* __restrict__ perm_slot, int32_t* __restrict__ row_of) {
+    __shared__ uint32_t mask[kMaxE][kPermBlockTokens / 32];
+    for (int i = threadIdx.x; i < E * (kPermBlockTokens / 32); i += blockDim.x) (&mask[0][0])[i] = 0;
+    __syncthreads();
+    const int tt = threadIdx.x;
+    const int64_t t = (int64_t)blockIdx.x * kPermBlockTokens + tt;
+    if (t < T)
+        for (int j = 0; j < k; ++j) atomicOr(&mask[topk_idx[t * k + j]][tt >> 5], 1u << (tt & 31));
+    __syncthreads();
+    if (t >= T) return;
+    for (int j = 0; j < k; ++j) {
+        const int e = topk_idx[t * k + j];
+        int rank = __popc(mask[e][tt >> 5] & ((1u << (tt & 31)) - 1u));
+        for (int w = 0; w < (tt >> 5); ++w) rank += __popc(mask[e][w]);
+        const int32_t row = blk_base[(int64_t)blockIdx.x * E + e] + rank;
+        perm_tok[row] = (int32_t)t;
+        perm_slot[row] = j;
+        row_of[t * k + j] = row;
+    }
+}
+
+int launch_perm_scatter(const int32_t* topk_idx, int64_t T, int32_t E, int32_t k, const int32_t* blk_base,
+                        int32_t* perm_tok, int32_t* perm_slot, int32_t* row_of, cudaStream_t st) {
+    const int64_t nblk = (T + kPermBlockTokens - 1) / kPermBlockTokens;
+    perm_scatter_kernel<<<(unsigned)nblk, kPermBlockTokens, 0, st>>>(topk_idx, T, E, k, blk_base, perm_tok,
+                                                                      perm_slot, row_of);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+}
+
+// ---- combine ---------------------------------------------------------------
+template <typename OutT>
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ d, const float* __restrict__ w,
+                                                      const int32_t* __restrict__ row_of, int64_t T, int32_t k,
+                                                      int64_t N, OutT* __restrict__ y) {
+    const int64_t n4 = N / 4;
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= T * n4) return;
+    const int64_t t = i / n4, c = (i % n4) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+        const float wj = w[t * k + j];
+        const float4 v = *reinterpret_cast<const float4*>(d + (int64_t)row_of[t * k + j] * N + c);
+        acc.x = fmaf(wj, v.x, acc.x);
+        acc.y = fmaf(wj, v.y, acc.y);
+        acc.z = fmaf(wj, v.z, acc.z);
+        acc.w = fmaf(wj, v.w, acc.w);
+    }
+    store_out<OutT>(y + t * N + c, acc.x);
+    store_out<OutT>(y + t * N + c + 1, acc.y);
+    store_out<OutT>(y + t * N + c + 2, acc.z);
+    store_out<OutT>(y + t * N + c + 3, acc.w);
+}
+
+int launch_combine(const float* d, const float* topk_w, const int32_t* row_of, int64_t T, int32_t k, int64_t N,
+                   void* y, int y_dtype, cudaStream_t st) {
+    const int64_t n = T * (N / 4);
+    const unsigned grid = (unsigned)((n + 255) / 256);
+    if (y_dtype == NVFP4_DTYPE_BF16)
+        combine_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(d, topk_w, row_of, T, k, N, (__nv_bfloat16*)y);
+    else
+        combine_kernel<float><<<grid, 256, 0, st>>>(d, topk_w, row_of, T, k, N, (float*)y);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,220 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4, the NVFP4 linear layer for B200 (sm_100a).
+ *
+ * The layer: a linear y = x W^T whose weight W [N, K] is stored as NVFP4, i.e.
+ * E2M1 4-bit codes, one E4M3 scale per 16 consecutive values along K and one
+ * fp32 scale per tensor:
+ *
+ *     W[n, k] = E2M1(code[n, k]) * E4M3(scale[n, k / 16]) * gs
+ *
+ * The pages this library follows name the format and the ways the layer runs,
+ * but do not define either:
+ *   - imp home page, "How does it work?": weights stay NVFP4 and the GPU
+ *     multiplies in that format instead of unpacking to 16 bits;
+ *   - Ignis README, "The decode round": decode linears are weight streaming at
+ *     the card's bandwidth (the W4A16 decode path here);
+ *   - Ignis README, "How fast" and "Credits": prefill in 2,048-token chunks,
+ *     split-K prefill, attention on FP4 tensor cores (the W4A4 prefill path);
+ *   - imp v0.20.0 release notes, "Highlights": a first-party NVFP4 quantizer
+ *     (nvfp4_quantize);
+ *   - CHImp Alpha v1.0 model card, "How it fits on one GPU": every token is
+ *     routed to 10 of 512 experts per layer and only those experts' weights
+ *     are read (moe_route_topk, moe_grouped_linear);
+ *   - Ignis README, "What sets it apart" / "Building it": a flat,
+ *     device-resident, step-level C ABI under a per-request error boundary
+ *     (the style of this header).
+ *
+ * Conventions for every call below.
+ *   - Every pointer argument is a DEVICE pointer (unless stated) owned by the
+ *     caller; the library keeps no reference after the call returns.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL means the legacy default stream).  No call allocates or frees
+ *     memory or synchronizes, except nvfp4_read_device_status.
+ *   - Every call validates its arguments on the host before launching any
+ *     kernel.  A call that returns an error has launched nothing and written
+ *     nothing.  Values behind device pointers (e.g. a per-tensor scale) are not
+ *     validated: they must be finite, and scales positive.
+ *   - Data pointers must be 16-byte aligned.
+ *   - Matrices are row-major.  Codes are packed two per byte, element 2j in
+ *     the low nibble of byte j.  Scale bytes are raw E4M3 with sign bit 0.
+ *   - Returns NVFP4_OK (0) or one of the NVFP4_ERR_* codes.
+ *
+ * Numerics.  W4A16 accumulates in fp32: per 16-element block, sum x * E2M1,
+ * then multiply by the block's E4M3 scale, then by gs at the end.  The
+ * tensor-core skinny path rounds activations to fp16 after a per-row
+ * power-of-two prescale (exact for every element within 2^32 of its row's
+ * largest magnitude).  W4A4 quantizes activations with the same rules as
+ * nvfp4_quantize and accumulates E2M1 x E2M1 products in fp32 on the tensor
+ * cores.  bf16 outputs are rounded to nearest even from fp32.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_NULL = 1,           /* a required pointer is NULL                   */
+    NVFP4_ERR_SHAPE = 2,          /* a size is out of range / not a multiple      */
+    NVFP4_ERR_ALIGN = 3,          /* a pointer is not 16-byte aligned             */
+    NVFP4_ERR_DTYPE = 4,          /* unsupported dtype code                       */
+    NVFP4_ERR_WORKSPACE = 5,      /* ws is NULL or ws_bytes below the query value */
+    NVFP4_ERR_ARCH = 6,           /* the current device is not sm_100             */
+    NVFP4_ERR_LAUNCH = 7,         /* a kernel launch or driver call failed        */
+    NVFP4_ERR_LAYOUT = 8,         /* scale layout not accepted by the chosen mode */
+    NVFP4_ERR_MODE = 9,           /* unknown mode or epilogue code                */
+    NVFP4_ERR_DEVICE_TIMEOUT = 10 /* a kernel's bounded wait ran out (read with
+                                     nvfp4_read_device_status)                    */
+};
+
+/* ---- enumerations ------------------------------------------------------ */
+enum { NVFP4_DTYPE_F32 = 0, NVFP4_DTYPE_BF16 = 1 };
+
+/* Scale layouts.
+ *   ROWMAJOR: scale (r, c) at byte r * (cols/16) + c.  rows * cols/16 bytes.
+ *   TILED:    the tensor-core scale-factor layout.  Rows are padded to
+ *             Rp = ceil(rows/128)*128 and scale columns to Cp = ceil((cols/16)/4)*4;
+ *             the matrix is cut into 128 x 4 atoms of 512 bytes, atoms ordered
+ *             with the column index fastest:
+ *               byte(r, c) = ((r/128) * (Cp/4) + c/4) * 512
+ *                            + (r%32) * 16 + ((r%128)/32) * 4 + (c%4).
+ *             Rp * Cp bytes; padding bytes are written as 0 by nvfp4_quantize.
+ *             This is the operand layout of tcgen05 block-scaled MMA, so a
+ *             128-row x 64-column tile's scales are one contiguous 512 B atom. */
+enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_TILED = 1 };
+
+/* Modes of the linear.  AUTO picks W4A16 for M <= 32 and W4A4 above. */
+enum { NVFP4_MODE_AUTO = 0, NVFP4_MODE_W4A16 = 1, NVFP4_MODE_W4A4 = 2 };
+
+/* Epilogues of moe_grouped_linear. */
+enum { NVFP4_EPI_NONE = 0, NVFP4_EPI_SWIGLU = 1, NVFP4_EPI_COMBINE = 2 };
+
+/* ---- helpers ------------------------------------------------------------ */
+
+/* Text of a status code (static storage). */
+const char* nvfp4_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int nvfp4_version(void);
+
+/* Bytes of a [rows, cols] tensor's scales in `sf_layout` (0 on bad arguments). */
+size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int sf_layout);
+
+/* Debug helper.  Copies the library's device status word (set by a kernel
+ * whose bounded wait ran out) into *status_out, resets it to NVFP4_OK, and
+ * synchronizes `stream`.  The only call that synchronizes. */
+int nvfp4_read_device_status(void* stream, int* status_out);
+
+/* ---- nvfp4_quantize ------------------------------------------------------
+ * NVFP4 quantization (imp v0.20.0 release notes, "Highlights": first-party
+ * NVFP4 quantizer, round-to-nearest part).  For x [rows, cols]:
+ *     gs      = *gs_in if gs_in != NULL, else amax(|x|) / 2688 (1.0 if amax == 0)
+ *     s[r, b] = E4M3(amax_b / (gs * 6))               (binary32: denom = gs * 6)
+ *     c[r, k] = E2M1(x[r, k] / (E4M3value(s) * gs))  (binary32 division)
+ * Rounding is to nearest with ties to the even code, saturating at 448 / 6,
+ * and keeps the sign (a negative value that rounds to 0 gives code 8).
+ * A block whose E4M3value(s) * gs is 0 stores +0 codes.
+ *   x       [rows, cols] in x_dtype (F32 or BF16)
+ *   gs_in   device float or NULL
+ *   codes   out, rows * cols/2 bytes
+ *   scales  out, nvfp4_scales_bytes(rows, cols, sf_layout) bytes
+ *   gs_out  out, one device float (the gs used)
+ *   ws      scratch of nvfp4_quantize_workspace(rows, cols) bytes (holds the
+ *           amax reduction); contents on entry are ignored.
+ * Requires cols % 16 == 0, rows >= 1. */
+size_t nvfp4_quantize_workspace(int64_t rows, int64_t cols);
+int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t cols,
+                   const float* gs_in, int sf_layout,
+                   uint8_t* codes, uint8_t* scales, float* gs_out,
+                   void* ws, size_t ws_bytes, void* stream);
+
+/* ---- nvfp4_linear --------------------------------------------------------
+ * y[m, n] = sum_k x[m, k] * W[n, k], W NVFP4 as above (Ignis README, "The
+ * decode round"; imp home page, "How does it work?").
+ *   x        [M, K] bf16 (x_dtype must be NVFP4_DTYPE_BF16)
+ *   w_codes  [N, K/2] bytes;  w_scales in w_sf_layout;  w_gs one device float
+ *   y        [M, N] in y_dtype (F32 or BF16)
+ *   mode     W4A16: weight-only, activations stay bf16.  Accepts either
+ *                   scale layout.  Any M >= 1.
+ *            W4A4:  activations quantized per call to NVFP4 (per-tensor gs,
+ *                   same rules as nvfp4_quantize), tcgen05 block-scaled MMA.
+ *                   Requires w_sf_layout == TILED and K % 256 == 0.
+ *            AUTO:  W4A16 if M <= 32, else W4A4.
+ *   ws       scratch of nvfp4_linear_workspace(M, K, N, mode) bytes (the
+ *            quantized activations for W4A4, the fp16 activations for the
+ *            tensor-core W4A16 path); contents on entry are ignored.
+ * Requires K % 16 == 0, M, N >= 1. */
+size_t nvfp4_linear_workspace(int64_t M, int64_t K, int64_t N, int mode);
+int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K,
+                 const uint8_t* w_codes, const uint8_t* w_scales, int w_sf_layout,
+                 const float* w_gs, int64_t N,
+                 void* y, int y_dtype, int mode,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/* ---- moe_route_topk ------------------------------------------------------
+ * Router of a routed mixture-of-experts layer (CHImp Alpha v1.0 model card,
+ * "How it fits on one GPU": 10 of 512 experts per token).
+ *     l[t, e]   = sum_h h[t, h] * Wr[e, h] (+ logit_bias[e]), fp32 accumulate
+ *     topk_idx  the k largest logits per token, equal logits -> lower index,
+ *               slots in descending logit order
+ *     topk_w    softmax over the k selected logits (= full softmax
+ *               renormalised over the top k)
+ *     expert_offsets[E+1]  exclusive prefix sum of per-expert counts
+ *     perm_tok[r], perm_slot[r]  the (token, slot) of row r, rows grouped by
+ *               expert ascending, tokens ascending within an expert
+ *     row_of[t*k + j]  the row of token t's slot j (inverse of the above)
+ *   h [T, H] bf16;  w_router [E, H] bf16;  logit_bias [E] fp32 or NULL;
+ *   logits_out [T, E] fp32 or NULL;  topk_idx, row_of [T, k] int32;
+ *   topk_w [T, k] fp32;  perm_tok, perm_slot [T*k] int32;
+ *   ws  scratch of moe_route_topk_workspace(T, E, k) bytes (per-expert
+ *       counters); contents on entry are ignored.
+ * Requires 1 <= k <= 32, k <= E <= 1024, H % 8 == 0, T >= 1. */
+size_t moe_route_topk_workspace(int64_t T, int32_t E, int32_t k);
+int moe_route_topk(const void* h, const void* w_router, const float* logit_bias,
+                   int64_t T, int64_t H, int32_t E, int32_t k,
+                   float* logits_out, int32_t* topk_idx, float* topk_w,
+                   int32_t* expert_offsets, int32_t* perm_tok, int32_t* perm_slot,
+                   int32_t* row_of, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- moe_grouped_linear --------------------------------------------------
+ * Expert linears over the permuted rows (CHImp, same section: only the chosen
+ * experts' weights are read).  For each expert e and row r in
+ * [expert_offsets[e], expert_offsets[e+1]):
+ *     out[r, :] = xin(r) @ W_e^T,  xin(r) = x[perm_tok[r]] if gather else x[r]
+ * then the epilogue:
+ *     NONE     y[r, n]  = out[r, n]                               y [R, N]
+ *     SWIGLU   y[r, j]  = silu(out[r, j]) * out[r, N/2 + j]        y [R, N/2]
+ *              (gate = first half of W_e's rows, up = second half)
+ *     COMBINE  y[t, n]  = sum_{j<k} topk_w[t, j] * out[row_of[t, j], n],
+ *              j ascending                                          y [R/k, N]
+ *   x        [rows of x, K] bf16 (x_dtype BF16)
+ *   w_codes  [E, N, K/2];  w_scales: E consecutive per-expert scale blocks of
+ *            nvfp4_scales_bytes(N, K, w_sf_layout) bytes;  w_gs [E] fp32
+ *   R        total rows (= T * k for routed input)
+ *   topk_w, row_of, k: used by COMBINE only (may be NULL / 0 otherwise)
+ *   y_dtype  F32 or BF16
+ *   mode     as nvfp4_linear (W4A16 / W4A4 / AUTO by R <= 32 * k ... see
+ *            moe_grouped_linear_workspace); W4A4 requires TILED scales.
+ *   ws       scratch of moe_grouped_linear_workspace(...) bytes.
+ * Experts with no rows are skipped: their weights are not read. */
+size_t moe_grouped_linear_workspace(int64_t R, int64_t K, int64_t N, int32_t E, int32_t k,
+                                    int epilogue, int mode);
+int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather,
+                       const int32_t* expert_offsets, const int32_t* perm_tok,
+                       int32_t E, int64_t R,
+                       const uint8_t* w_codes, const uint8_t* w_scales, int w_sf_layout,
+                       const float* w_gs, int64_t N,
+                       int epilogue, const float* topk_w, const int32_t* row_of, int32_t k,
+                       void* y, int y_dtype, int mode,
+                       void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_H */

@@ -1,0 +1,145 @@
+"""The C-ABI library: exported symbols and host-side validation (no GPU needed).
+
+Every entry point validates its arguments on the host before touching the
+device, so these tests call it with fake (but aligned) pointers and check the
+status codes; nothing is launched.  A fully valid call on a machine without a
+B200 must return NVFP4_ERR_ARCH instead of launching.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import bit_linear_moe_b200 as nv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = ctypes.c_void_p(0x10000)           # aligned, never dereferenced
+FAKE2 = ctypes.c_void_p(0x20000)
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_linear_moe_b200 import build
+    build.build()
+    return nv.lib()
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared_functions()
+    assert "nvfp4_linear" in names and "moe_grouped_linear" in names and len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for s in range(11):
+        assert nv.status_string(s) not in ("", "unknown status")
+    assert nv.status_string(99) == "unknown status"
+
+
+def test_scales_bytes(L):
+    assert nv.nvfp4_scales_bytes(5, 48, nv.SF_ROWMAJOR) == 15
+    assert nv.nvfp4_scales_bytes(5, 48, nv.SF_TILED) == 128 * 4
+    assert nv.nvfp4_scales_bytes(129, 1024, nv.SF_TILED) == 256 * 64
+    assert nv.nvfp4_scales_bytes(5, 40, nv.SF_TILED) == 0
+
+
+def _linear(L, **kw):
+    a = dict(x=FAKE, xd=nv.DTYPE_BF16, M=1, K=64, c=FAKE, s=FAKE, lay=nv.SF_ROWMAJOR, gs=FAKE, N=16,
+             y=FAKE2, yd=nv.DTYPE_F32, mode=nv.MODE_W4A16, ws=None, wsb=0)
+    a.update(kw)
+    return L.nvfp4_linear(a["x"], a["xd"], a["M"], a["K"], a["c"], a["s"], a["lay"], a["gs"], a["N"], a["y"],
+                          a["yd"], a["mode"], a["ws"], a["wsb"], None)
+
+
+def test_linear_validation(L):
+    assert _linear(L, x=None) == nv.ERR_NULL
+    assert _linear(L, K=40) == nv.ERR_SHAPE
+    assert _linear(L, M=0) == nv.ERR_SHAPE
+    assert _linear(L, N=0) == nv.ERR_SHAPE
+    assert _linear(L, c=MISALIGNED) == nv.ERR_ALIGN
+    assert _linear(L, xd=nv.DTYPE_F32) == nv.ERR_DTYPE
+    assert _linear(L, yd=7) == nv.ERR_DTYPE
+    assert _linear(L, lay=5) == nv.ERR_LAYOUT
+    assert _linear(L, mode=9) == nv.ERR_MODE
+    if not torch.cuda.is_available():
+        assert _linear(L) == nv.ERR_ARCH
+
+
+def test_linear_w4a4_validation(L):
+    ws_need = L.nvfp4_linear_workspace(512, 1024, 256, nv.MODE_W4A4)
+    assert ws_need > 512 * 512
+    assert _linear(L, M=512, K=1024, N=256, mode=nv.MODE_W4A4, lay=nv.SF_ROWMAJOR,
+                   ws=FAKE, wsb=ws_need) == nv.ERR_LAYOUT
+    assert _linear(L, M=512, K=1000 + 8, N=256, mode=nv.MODE_W4A4, lay=nv.SF_TILED,
+                   ws=FAKE, wsb=ws_need) == nv.ERR_SHAPE
+    assert _linear(L, M=512, K=1024, N=256, mode=nv.MODE_W4A4, lay=nv.SF_TILED,
+                   ws=FAKE, wsb=ws_need - 1) == nv.ERR_WORKSPACE
+
+
+def test_quantize_validation(L):
+    def q(**kw):
+        a = dict(x=FAKE, xd=nv.DTYPE_F32, rows=4, cols=64, gs=None, lay=nv.SF_ROWMAJOR, c=FAKE, s=FAKE,
+                 go=FAKE2, ws=FAKE2, wsb=256)
+        a.update(kw)
+        return L.nvfp4_quantize(a["x"], a["xd"], a["rows"], a["cols"], a["gs"], a["lay"], a["c"], a["s"],
+                                a["go"], a["ws"], a["wsb"], None)
+    assert q(x=None) == nv.ERR_NULL
+    assert q(cols=24) == nv.ERR_SHAPE
+    assert q(rows=0) == nv.ERR_SHAPE
+    assert q(wsb=16) == nv.ERR_WORKSPACE
+    assert q(ws=None) == nv.ERR_WORKSPACE
+    assert q(s=MISALIGNED) == nv.ERR_ALIGN
+    assert q(xd=3) == nv.ERR_DTYPE
+    assert q(lay=2) == nv.ERR_LAYOUT
+    if not torch.cuda.is_available():
+        assert q() == nv.ERR_ARCH
+
+
+def test_route_validation(L):
+    def r(**kw):
+        a = dict(h=FAKE, w=FAKE, b=None, T=4, H=64, E=16, k=4, lo=None, ws=FAKE2)
+        a.update(kw)
+        wsb = a.pop("wsb", L.moe_route_topk_workspace(a["T"], a["E"], a["k"]))
+        return L.moe_route_topk(a["h"], a["w"], a["b"], a["T"], a["H"], a["E"], a["k"], a["lo"], FAKE, FAKE,
+                                FAKE, FAKE, FAKE, FAKE, a["ws"], wsb, None)
+    assert r(h=None) == nv.ERR_NULL
+    assert r(k=0) == nv.ERR_SHAPE
+    assert r(k=17, E=16) == nv.ERR_SHAPE
+    assert r(E=2048) == nv.ERR_SHAPE
+    assert r(H=60) == nv.ERR_SHAPE
+    assert r(wsb=8) == nv.ERR_WORKSPACE
+    if not torch.cuda.is_available():
+        assert r() == nv.ERR_ARCH
+
+
+def test_grouped_validation(L):
+    def g(**kw):
+        a = dict(x=FAKE, K=64, gather=1, off=FAKE, pt=FAKE, E=8, R=16, c=FAKE, s=FAKE, lay=nv.SF_ROWMAJOR,
+                 gs=FAKE, N=32, epi=nv.EPI_NONE, tw=None, ro=None, k=0, y=FAKE2, mode=nv.MODE_W4A16)
+        a.update(kw)
+        wsb = L.moe_grouped_linear_workspace(a["R"], a["K"], a["N"], a["E"], a["k"], a["epi"], a["mode"])
+        return L.moe_grouped_linear(a["x"], nv.DTYPE_BF16, a["K"], a["gather"], a["off"], a["pt"], a["E"],
+                                    a["R"], a["c"], a["s"], a["lay"], a["gs"], a["N"], a["epi"], a["tw"],
+                                    a["ro"], a["k"], a["y"], nv.DTYPE_F32, a["mode"], FAKE2 if wsb else None,
+                                    wsb, None)
+    assert g(pt=None) == nv.ERR_NULL
+    assert g(epi=nv.EPI_COMBINE) == nv.ERR_NULL
+    assert g(epi=nv.EPI_COMBINE, tw=FAKE, ro=FAKE, k=3) == nv.ERR_SHAPE
+    assert g(epi=nv.EPI_SWIGLU, N=33) == nv.ERR_SHAPE
+    assert g(epi=7) == nv.ERR_MODE
+    if not torch.cuda.is_available():
+        assert g() == nv.ERR_ARCH
