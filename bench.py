@@ -40,6 +40,8 @@ METRIC = "NVFP4 linear: decode GB/s (% HBM peak); prefill TFLOPS (% FP4 tensor p
 SHAPES = (("qkv", 5120, 10240, 1), ("o_proj", 5120, 5120, 2), ("gate_up", 5120, 34816, 3),
           ("down", 17408, 5120, 4))
 FALLBACK_HBM_GBS = 6650.0
+WORKLOAD = ("dense27b decode linears (QKV 5120x10240, o_proj 5120x5120, gate_up 5120x34816, down 17408x5120), "
+            "W4A16, M=1")
 
 
 def decode_bytes(M, K, N):
@@ -150,36 +152,62 @@ def run_native(args, rank, world, dist):
         layers.append((name, K, N, copies, x, y))
     torch.cuda.synchronize()
 
-    def step(i, events=None):
-        for j, (name, K, N, copies, x, y) in enumerate(layers):
-            c, s, g = copies[i % 2]
-            if events is not None:
-                events[j][0].record(stream)
-            nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16)
-            if events is not None:
-                events[j][1].record(stream)
+    ws = {}
+    for name, K, N, copies, x, y in layers:
+        nbytes = int(nv.lib().nvfp4_linear_workspace(1, K, N, nv.MODE_W4A16))
+        ws[name] = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev) if nbytes else None
+
+    def call(j, i):
+        name, K, N, copies, x, y = layers[j]
+        c, s, g = copies[i % 2]
+        nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16, ws=ws[name])
+
+    def step(i):
+        for j in range(len(layers)):
+            call(j, i)
 
     step_bytes = sum(decode_bytes(1, K, N) for _, K, N, *_ in layers)
 
-    for i in range(args.warmup):
+    # eager warm-up (kernel attributes, cluster-size choice), then capture:
+    # one graph per weight copy for the whole step, one per (shape, copy)
+    for i in range(3):
         step(i)
     torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    per_launch = [[] for _ in layers]
-    ev_all = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in layers] for _ in range(args.steps)]
+    side = torch.cuda.Stream(device=dev)
+    side.wait_stream(stream)
+    step_graphs, shape_graphs = [], []
+    with torch.cuda.stream(side):
+        for i in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                step(i)
+            step_graphs.append(g)
+        for j in range(len(layers)):
+            pair = []
+            for i in range(2):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=side):
+                    call(j, i)
+                pair.append(g)
+            shape_graphs.append(pair)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev.index) as clk:
+        time.sleep(0.5)
+        for i in range(args.warmup):
+            step_graphs[i % 2].replay()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
         torch.cuda.synchronize()
         t0.record(stream)
         for i in range(args.steps):
-            step(i, ev_all[i])
+            step_graphs[i % 2].replay()
         t1.record(stream)
         torch.cuda.synchronize()
     ms = t0.elapsed_time(t1)
-    for i in range(args.steps):
-        for j in range(len(layers)):
-            per_launch[j].append(ev_all[i][j][0].elapsed_time(ev_all[i][j][1]))
     if dist:
         t = torch.tensor([ms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -187,15 +215,26 @@ def run_native(args, rank, world, dist):
     ms_per_step = ms / args.steps
     value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
 
+    # per-shape device time: each linear alone, replayed from its graph
+    reps = max(200, min(2000, args.steps))
+    per_shape, launch_ms = {}, 0.0
+    for j, (name, K, N, *_) in enumerate(layers):
+        for i in range(4):
+            shape_graphs[j][i % 2].replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(reps):
+            shape_graphs[j][i % 2].replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        m = a.elapsed_time(b) / reps
+        launch_ms += m
+        per_shape[name] = {"us": round(m * 1e3, 2), "GB/s": round(decode_bytes(1, K, N) / (m * 1e-3) / 1e9, 1)}
+
     # roofline of the dominant kernel (the W4A16 decode kernel: every launch)
     peak, peak_kind = load_peaks()
-    launch_ms = sum(sum(v) for v in per_launch) / args.steps
     achieved = step_bytes / (launch_ms * 1e-3) / 1e9
-    per_shape = {}
-    for (name, K, N, *_), v in zip(layers, per_launch):
-        m = statistics.median(v)
-        per_shape[name] = {"us": round(m * 1e3, 2), "GB/s": round(decode_bytes(1, K, N) / (m * 1e-3) / 1e9, 1)}
-    traffic = kernel_traffic("gemv.cu", "gemv_w4a16_decode")
+    traffic = kernel_traffic("gemv_tma.cu", "gemv_tma_decode")
 
     # end to end through the public API: pinned host x in, host y out, every step
     xh = [torch.empty((1, K), dtype=torch.bfloat16).pin_memory() for _, K, *_ in layers]
@@ -209,7 +248,7 @@ def run_native(args, rank, world, dist):
         for j, (name, K, N, copies, x, y) in enumerate(layers):
             c, s, g = copies[i % 2]
             x.copy_(xh[j], non_blocking=True)
-            nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16)
+            nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16, ws=ws[name])
             yh[j].copy_(y, non_blocking=True)
 
     for i in range(args.warmup):
@@ -239,14 +278,13 @@ def run_native(args, rank, world, dist):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 weights x bf16 activations, fp32 accumulate",
         "data": "synthetic: weights N(0,0.02) fp32 quantized on device, activations N(0,1) bf16",
-        "config": {"workload": "dense27b decode linears (QKV 5120x10240, o_proj 5120x5120, gate_up 5120x34816, "
-                               "down 17408x5120), W4A16, M=1",
-                   "M": 1, "bytes_per_step": step_bytes,
+        "config": {"workload": WORKLOAD, "M": 1, "bytes_per_step": step_bytes,
+                   "timing": "CUDA-graph replay of the step (4 linears), events on the launching stream",
                    "l2": "weights rotated over 2 copies (389 MB) > 126 MB L2",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
-                     "kernel": "gemv_w4a16_kernel (4 launches per step, CUDA events per launch)"},
+                     "kernel": "gemv_tma_kernel (the only launch of each linear): per-shape graph replays timed with CUDA events"},
         "e2e": {"value": round(e2e, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 4 * args.steps,
         "clocks": clk.summary(),
@@ -255,30 +293,44 @@ def run_native(args, rank, world, dist):
     return line
 
 
-def decode_sweep(nv, torch, dev, layers, reps=20):
-    """Median per-launch GB/s for each shape and M (weights rotated over 2 copies)."""
+def decode_sweep(nv, torch, dev, layers, reps=200):
+    """Per-launch GB/s for each shape and M, from CUDA-graph replays (weights
+    rotated over 2 copies)."""
     from bit_linear_moe_b200 import synth
     out = {}
     stream = torch.cuda.current_stream()
+    side = torch.cuda.Stream(device=dev)
     for name, K, N, copies, _, _ in layers:
+        seed = dict((s[0], s[3]) for s in SHAPES)[name]
         row = {}
         for M in synth.DECODE_M:
-            x = torch.from_numpy(synth.decode_x(SHAPES[[s[0] for s in SHAPES].index(name)][3], M, K)).to(
-                torch.bfloat16).to(dev)
+            x = torch.from_numpy(synth.decode_x(seed, M, K)).to(torch.bfloat16).to(dev)
             y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            nbytes = int(nv.lib().nvfp4_linear_workspace(M, K, N, nv.MODE_W4A16))
+            ws = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
             for i in range(3):
                 c, s, g = copies[i % 2]
-                nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16)
-            ts = []
-            for i in range(reps):
-                c, s, g = copies[i % 2]
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16)
-                b.record(stream)
-                ts.append((a, b))
+                nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16, ws=ws)
             torch.cuda.synchronize()
-            m = statistics.median(a.elapsed_time(b) for a, b in ts)
+            side.wait_stream(stream)
+            graphs = []
+            with torch.cuda.stream(side):
+                for i in range(2):
+                    gr = torch.cuda.CUDAGraph()
+                    c, s, g = copies[i]
+                    with torch.cuda.graph(gr, stream=side):
+                        nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16, ws=ws)
+                    graphs.append(gr)
+            stream.wait_stream(side)
+            for i in range(4):
+                graphs[i % 2].replay()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(reps):
+                graphs[i % 2].replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            m = a.elapsed_time(b) / reps
             row[str(M)] = round(decode_bytes(M, K, N) / (m * 1e-3) / 1e9, 1)
         out[name] = row
     return out
@@ -286,37 +338,61 @@ def decode_sweep(nv, torch, dev, layers, reps=20):
 
 # --------------------------------------------------------------- reference ----
 
-def oracle_decode_sample(reps: int = 1):
+def oracle_decode_sample(min_seconds: float = 10.0, row_frac: int = 1):
     """Time the oracle's W4A16 linear on the same four shapes at M = 1 (weights
-    quantized by the oracle outside the timed region).  Returns (GB/s, seconds, threads)."""
+    quantized by the oracle outside the timed region), repeating the four
+    linears until ``min_seconds`` have passed.  ``row_frac`` > 1 keeps every
+    row_frac-th weight row (a bounded sample).  Returns (GB/s, seconds, passes, threads)."""
     import oracle
     from bit_linear_moe_b200 import synth
     qs = []
     for name, K, N, seed in SHAPES:
-        q = oracle.quantize(synth.dense_weight(seed, K, N))
-        qs.append((K, N, q, synth.decode_x(seed, 1, K)))
+        c, s_, g = oracle.quantize(synth.dense_weight(seed, K, N)[::row_frac])
+        qs.append((K, c.shape[0], (c, s_, g), synth.decode_x(seed, 1, K)))
     t = time.perf_counter()
-    nbytes = 0
-    for _ in range(reps):
+    nbytes, passes = 0, 0
+    while True:
         for K, N, q, x in qs:
             oracle.linear_w4a16(x, *q)
             nbytes += decode_bytes(1, K, N)
-    dt = time.perf_counter() - t
-    return nbytes / dt / 1e9, dt, oracle.num_threads()
+        passes += 1
+        dt = time.perf_counter() - t
+        if dt >= min_seconds:
+            break
+    return nbytes / dt / 1e9, dt, passes, oracle.num_threads()
 
 
 def run_reference(args):
-    gbs, dt, threads = oracle_decode_sample(reps=1)
-    step_s = dt
+    """The oracle as the reference arm: each step is the four linears at M = 1
+    over every 64th weight row (a bounded sample of the workload)."""
+    import oracle
+    from bit_linear_moe_b200 import synth
+    qs = []
+    for name, K, N, seed in SHAPES:
+        c, s_, g = oracle.quantize(synth.dense_weight(seed, K, N)[::64])
+        qs.append((K, c.shape[0], (c, s_, g), synth.decode_x(seed, 1, K)))
+    step_bytes = sum(decode_bytes(1, K, N) for K, N, _, _ in qs)
+
+    def step():
+        for K, N, q, x in qs:
+            oracle.linear_w4a16(x, *q)
+
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t
+    gbs = step_bytes * args.steps / dt / 1e9
+    sample = "each step: the four linears at M=1 over every 64th weight row"
     line = {
         "impl": "reference", "metric": METRIC, "value": round(gbs, 3), "unit": "GB/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 2),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp64 accumulate (CPU oracle)",
         "data": "synthetic, same generator as the native arm",
-        "config": {"workload": "dense27b decode linears (QKV 5120x10240, o_proj 5120x5120, gate_up 5120x34816, "
-                               "down 17408x5120), W4A16, M=1", "M": 1},
-        "cpu_baseline": {"value": round(gbs, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
-                         "sample": "one step = the four linears at M=1, timed once after oracle quantization"},
+        "config": {"workload": WORKLOAD, "M": 1},
+        "cpu_baseline": {"value": round(gbs, 3), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": round(gbs, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     return line
@@ -325,8 +401,8 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--quick", action="store_true", help="headline only (no sweeps, no CPU baseline)")
     args = ap.parse_args()
@@ -349,10 +425,10 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = tdist
     line = run_native(args, rank, world, dist)
-    if rank == 0 and not args.quick:
-        gbs, dt, threads = oracle_decode_sample(reps=1)
+    if rank == 0 and world == 1 and not args.quick:
+        gbs, dt, passes, threads = oracle_decode_sample(min_seconds=10.0)
         line["cpu_baseline"] = {"value": round(gbs, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
-                                "sample": f"the four linears at M=1 once ({dt:.1f} s)"}
+                                "sample": f"the four linears at M=1, full weights, {passes} passes in {dt:.1f} s"}
     if rank == 0:
         print(json.dumps(line))
     if dist:

@@ -11,6 +11,19 @@ namespace nvfp4 {
 __device__ int g_device_status = 0;
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Device address of the status word, looked up once per device.
+static int* device_status_ptr() {
+    static int* cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+        cache[dev] = (int*)p;
+    }
+    return cache[dev];
+}
 static size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
 
 // The current device must be sm_100 (B200 / GB200 class).  Cached per device.
@@ -39,6 +52,14 @@ static size_t scales_bytes(int64_t rows, int64_t cols, int layout) {
     if (layout == NVFP4_SF_TILED) return (size_t)((rows + 127) / 128 * 128) * (size_t)((nsf + 3) / 4 * 4);
     return 0;
 }
+
+// Grid limits of the W4A16 kernels (row tiles of >= 2 rows on grid.y, token
+// groups of <= 4 rows on grid.x).
+constexpr int64_t kMaxW4A16N = 65535 * 2;
+constexpr int64_t kMaxW4A16M = (int64_t)1 << 30;
+
+// W4A16 workspace: fp16 activations and one inverse scale per row.
+static size_t w4a16_ws(int64_t rows, int64_t K) { return align256((size_t)(rows * K) * 2) + align256((size_t)rows * 4); }
 
 // Row padding of a W4A4 operand: the tensor-core tiles are 128 rows.
 static int64_t moe_w4a4_rows(int64_t R, int32_t E) { return R + (int64_t)E * 127; }
@@ -128,7 +149,7 @@ size_t nvfp4_linear_workspace(int64_t M, int64_t K, int64_t N, int mode) {
         // amax word, gs, activation codes, tiled activation scales
         return align256(256) + align256((size_t)(M * K / 2)) + align256(scales_bytes(M, K, NVFP4_SF_TILED));
     }
-    return 0;
+    return decode_tma_supported(M, K, N) ? 0 : w4a16_ws(M, K);
 }
 
 int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t* w_codes, const uint8_t* w_scales,
@@ -146,14 +167,24 @@ int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t
     if (mode == NVFP4_MODE_W4A4) {
         if (w_sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_LAYOUT;
         if (K % 256) return NVFP4_ERR_SHAPE;
+    } else if (N > kMaxW4A16N || M > kMaxW4A16M) {
+        return NVFP4_ERR_SHAPE;
     }
     const size_t need = nvfp4_linear_workspace(M, K, N, mode);
     if (need && (!ws || ws_bytes < need)) return NVFP4_ERR_WORKSPACE;
     if (need && !aligned16(ws)) return NVFP4_ERR_ALIGN;
     NVFP4_TRY(check_arch());
     if (mode == NVFP4_MODE_W4A4) return NVFP4_ERR_MODE;  // tensor-core path not wired yet
+    cudaStream_t st = (cudaStream_t)stream;
+    if (decode_tma_supported(M, K, N))
+        return launch_decode_tma(x, M, K, w_codes, w_scales, w_sf_layout, w_gs, N, y, y_dtype, device_status_ptr(),
+                                 st);
+    void* xh = ws;
+    float* inv = (float*)((char*)ws + align256((size_t)(M * K) * 2));
+    NVFP4_TRY(launch_x_prep(x, nullptr, M, K, xh, inv, st));
     GemvArgs a{};
-    a.x = x;
+    a.xh = xh;
+    a.inv_scale = inv;
     a.M = M;
     a.K = K;
     a.codes = w_codes;
@@ -166,7 +197,7 @@ int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t
     a.y = y;
     a.y_dtype = y_dtype;
     a.ldy = N;
-    return launch_gemv_w4a16(a, (cudaStream_t)stream);
+    return launch_gemv_w4a16(a, st);
 }
 
 // ---- MoE routing -------------------------------------------------------------------
@@ -217,6 +248,7 @@ size_t moe_grouped_linear_workspace(int64_t R, int64_t K, int64_t N, int32_t E, 
     mode = resolve_grouped_mode(mode, R);
     size_t need = 0;
     if (epilogue == NVFP4_EPI_COMBINE) need += align256((size_t)(R * N) * 4);
+    if (mode == NVFP4_MODE_W4A16) need += w4a16_ws(R, K);
     if (mode == NVFP4_MODE_W4A4) {
         const int64_t rp = moe_w4a4_rows(R, E);
         need += align256(256) + align256((size_t)(rp * K / 2)) + align256(scales_bytes(rp, K, NVFP4_SF_TILED)) +
@@ -250,6 +282,8 @@ int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const 
     if (mode == NVFP4_MODE_W4A4) {
         if (w_sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_LAYOUT;
         if (K % 256) return NVFP4_ERR_SHAPE;
+    } else if (K % 32 || N > kMaxW4A16N) {
+        return NVFP4_ERR_SHAPE;
     }
     const size_t need = moe_grouped_linear_workspace(R, K, N, E, k, epilogue, mode);
     if (need && (!ws || ws_bytes < need)) return NVFP4_ERR_WORKSPACE;
@@ -257,9 +291,18 @@ int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const 
     NVFP4_TRY(check_arch());
     if (mode == NVFP4_MODE_W4A4) return NVFP4_ERR_MODE;  // tensor-core path not wired yet
     cudaStream_t st = (cudaStream_t)stream;
+    char* wp = (char*)ws;
+    float* d = nullptr;
+    if (epilogue == NVFP4_EPI_COMBINE) {
+        d = (float*)wp;
+        wp += align256((size_t)(R * N) * 4);
+    }
+    void* xh = wp;
+    float* inv = (float*)(wp + align256((size_t)(R * K) * 2));
+    NVFP4_TRY(launch_x_prep(x, gather ? perm_tok : nullptr, R, K, xh, inv, st));
     GemvArgs a{};
-    a.x = x;
-    a.gather = gather ? perm_tok : nullptr;
+    a.xh = xh;
+    a.inv_scale = inv;
     a.M = R;
     a.K = K;
     a.codes = w_codes;
@@ -271,7 +314,6 @@ int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const 
     a.offsets = expert_offsets;
     a.E = E;
     if (epilogue == NVFP4_EPI_COMBINE) {
-        float* d = (float*)ws;
         a.epilogue = NVFP4_EPI_NONE;
         a.y = d;
         a.y_dtype = NVFP4_DTYPE_F32;

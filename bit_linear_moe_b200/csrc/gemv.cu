@@ -1,56 +1,122 @@
 // K2: W4A16 linear on CUDA cores, for decode widths (Ignis README, "The decode
 // round": decode is weight streaming at the card's bandwidth).
 //
-// y[m, n] = gs * sum_b E4M3(s[n, b]) * sum_{k in block b} x[m, k] * E2M1(c[n, k])
+//   y[m, n] = gs * 2^-p_m * sum_b E4M3(s[n, b]) * sum_{k in b} xh[m, k] * E2M1(c[n, k])
 //
-// Work split: a warp owns R weight rows; its lanes stride over K in chunks of
-// 2*VB elements (VB = 16: one 128-bit load of 32 codes + one 16-bit load of
-// the two block scales per row).  The activation chunk is converted to fp32
-// once and reused for all R rows.  Per block: 16 FMAs into a block partial,
-// then one FMA by the block scale; gs is applied once at the end.  Lanes are
-// reduced with warp shuffles.  The weight stream uses non-allocating 128-bit
-// loads, so each weight byte crosses HBM once; activations come through the
-// read-only cache.
+// where xh = x * 2^p_m in fp16 (prepared once per call by x_prep_kernel; p_m
+// puts the row's largest magnitude in [2^14, 2^15), so xh equals x exactly
+// for every element within 2^28 of the row maximum).  Each weight pair is
+// unpacked by one cvt.rn.f16x2.e2m1x2 (exact) and multiplied with the
+// mixed-precision fma.rn.f32.f16 (exact product, fp32 accumulate): one
+// quarter-rate conversion per two elements and one FMA per element.  Per
+// 16-element block the partial sum is scaled once by the E4M3 block scale.
 //
-// Grid: x = token groups (dense) or experts (grouped), y = row tiles.  With
-// token groups fastest, the CTAs that read the same weight rows for different
-// token groups run together and share the rows through L2.
+// Work split: a CTA has 8 warps = RG row groups x QS K-splits.  A warp owns R
+// weight rows (2: the activation chunk it loads is reused for both) and one
+// K-split; its lanes stride over the split in 16-byte chunks (32 codes), and
+// all of the warp's chunk loads for a batch are issued before any of them is
+// consumed, so up to R*J 16-byte loads per lane are in flight.  Partial sums
+// of the QS splits meet in shared memory.  QS is picked per shape so that
+// small-N matrices still spread over all SMs.  The weight stream uses
+// non-allocating 128-bit loads; activations and scales go through L1.
 //
 // Grouped form (mixture of experts; CHImp Alpha v1.0 model card, "How it fits
-// on one GPU": only the chosen experts are read): expert e's rows are
-// [offsets[e], offsets[e+1]); an expert without rows exits before touching its
-// weights.  SWIGLU pairs weight row j (gate) with row N/2 + j (up) in the same
-// warp and writes silu(g) * u.
+// on one GPU": only the chosen experts are read): grid.x walks the experts,
+// expert e's rows are [offsets[e], offsets[e+1]); an expert without rows
+// exits before touching its weights.  SWIGLU gives a warp the gate row j and
+// the up row N/2 + j and writes silu(g) * u.
 #include "common.cuh"
 #include "internal.h"
 
 namespace nvfp4 {
 
-template <int VB>
-NVFP4_DEV void load_codes(const uint8_t* p, uint32_t (&w)[VB / 4]) {
-    if constexpr (VB == 16) {
-        uint4 v = ldg_stream(p);
-        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-    } else {
-        uint2 v;
-        asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-        w[0] = v.x; w[1] = v.y;
+// ---- activation prep: bf16 -> fp16 * 2^p per row ----------------------------
+__global__ void __launch_bounds__(256) x_prep_kernel(const __nv_bfloat16* __restrict__ x,
+                                                     const int32_t* __restrict__ gather, int64_t K,
+                                                     __half* __restrict__ xh, float* __restrict__ inv_scale) {
+    const int64_t m = blockIdx.x;
+    const __nv_bfloat16* xr = x + (gather ? (int64_t)gather[m] : m) * K;
+    float mx = 0.0f;
+    for (int64_t k = threadIdx.x * 8; k < K; k += blockDim.x * 8) {
+        const uint4 v = ldg_v4(xr + k);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mx = fmaxf(mx, fmaxf(fabsf(bf16lo_to_f32(u[j])), fabsf(bf16hi_to_f32(u[j]))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    __shared__ float red[8];
+    __shared__ float s_scale;
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < 8; ++w) mx = fmaxf(mx, red[w]);
+        // p = 14 - floor(log2(mx)) so that mx * 2^p lies in [2^14, 2^15)
+        int p = 0;
+        if (mx > 0.0f) p = 14 - (int)((__float_as_uint(mx) >> 23) & 0xFF) + 127;
+        p = p < -126 ? -126 : (p > 126 ? 126 : p);
+        s_scale = __uint_as_float((uint32_t)(127 + p) << 23);
+        inv_scale[m] = __uint_as_float((uint32_t)(127 - p) << 23);
+    }
+    __syncthreads();
+    const float sc = s_scale;
+    for (int64_t k = threadIdx.x * 8; k < K; k += blockDim.x * 8) {
+        const uint4 v = ldg_v4(xr + k);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __half2 h = __floats2half2_rn(bf16lo_to_f32(u[j]) * sc, bf16hi_to_f32(u[j]) * sc);
+            o[j] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(xh + m * K + k) = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
 
-template <int MT, int R, int VB, int LAYOUT, typename OutT, int EPI>
+// ---- main kernel ---------------------------------------------------------------
+
+NVFP4_DEV float fma_f16(uint16_t a, uint16_t b, float c) {
+    float d;
+    asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
+    return d;
+}
+
+// 32 products of one 16-byte code chunk with 32 fp16 activations, as two
+// block partials (elements 0..15 and 16..31).
+NVFP4_DEV void chunk_dot(const uint4& wq, const uint32_t (&xw)[16], float& p0, float& p1) {
+    const uint32_t w[4] = {wq.x, wq.y, wq.z, wq.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t h[4];
+        e2m1x8_to_f16x2(w[j], h);
+        float p = (j < 2) ? p0 : p1;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t xv = xw[4 * j + q];
+            p = fma_f16((uint16_t)(h[q] & 0xFFFF), (uint16_t)(xv & 0xFFFF), p);
+            p = fma_f16((uint16_t)(h[q] >> 16), (uint16_t)(xv >> 16), p);
+        }
+        if (j < 2) p0 = p; else p1 = p;
+    }
+}
+
+template <int MT, int R, int QS, int J, int LAYOUT, typename OutT, int EPI>
 __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
-    constexpr int CE = 2 * VB;          // elements per chunk
-    constexpr int NB = CE / 16;         // blocks per chunk
-    constexpr int RW = (EPI == NVFP4_EPI_SWIGLU) ? R / 2 : R;  // output columns per warp
+    constexpr int RG = 8 / QS;                                    // row groups per CTA
+    constexpr int RW = (EPI == NVFP4_EPI_SWIGLU) ? 1 : R;         // output columns per warp
+    static_assert(EPI != NVFP4_EPI_SWIGLU || R == 2, "SwiGLU pairs one gate and one up row");
+    __shared__ float red[8][R][MT];
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = warp / QS, q = warp % QS;
     const int64_t K = a.K;
-    const int64_t nchunk = K / CE;
+    const int64_t nch = K >> 5;                                   // 32-element chunks per row
     const int64_t nsf = K >> 4;
     const int64_t ncols_out = (EPI == NVFP4_EPI_SWIGLU) ? a.N / 2 : a.N;
+    const int64_t c_begin = nch * q / QS, c_end = nch * (q + 1) / QS;
 
-    const int64_t col0 = ((int64_t)blockIdx.y * 8 + warp) * RW;
-    if (col0 >= ncols_out) return;
+    const int64_t col0 = ((int64_t)blockIdx.y * RG + g) * RW;
+    const bool warp_active = col0 < ncols_out;
 
     int64_t row_begin, row_end;
     const uint8_t* codes = a.codes;
@@ -60,7 +126,7 @@ __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
         const int e = blockIdx.x;
         row_begin = a.offsets[e];
         row_end = a.offsets[e + 1];
-        if (row_end <= row_begin) return;  // untouched expert: its weights are never read
+        if (row_end <= row_begin) return;  // untouched expert: its weights are never read (CTA-uniform)
         codes += (int64_t)e * a.N * (K >> 1);
         scales += (int64_t)e * a.sf_stride;
         gs = a.gs[e];
@@ -70,152 +136,227 @@ __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
         gs = a.gs[0];
     }
 
-    // Weight rows of this warp (clamped; invalid ones are computed and dropped).
     int64_t wrow[R];
     bool cvalid[RW];
 #pragma unroll
     for (int i = 0; i < RW; ++i) {
         const int64_t c = col0 + i;
         cvalid[i] = c < ncols_out;
-        const int64_t cc = cvalid[i] ? c : col0;
+        const int64_t cc = cvalid[i] ? c : (warp_active ? col0 : 0);
         wrow[i] = cc;
-        if constexpr (EPI == NVFP4_EPI_SWIGLU) wrow[RW + i] = a.N / 2 + cc;
+        if constexpr (EPI == NVFP4_EPI_SWIGLU) wrow[1] = a.N / 2 + cc;
     }
 
-    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(a.x);
+    const __half* xh = reinterpret_cast<const __half*>(a.xh);
     for (int64_t m0 = row_begin; m0 < row_end; m0 += MT) {
         const int nt = (int)((row_end - m0) < MT ? (row_end - m0) : MT);
-        const __nv_bfloat16* xr[MT];
+        const __half* xr[MT];
 #pragma unroll
-        for (int t = 0; t < MT; ++t) {
-            const int64_t r = m0 + (t < nt ? t : 0);
-            const int64_t src = a.gather ? a.gather[r] : r;
-            xr[t] = xb + src * K;
-        }
+        for (int t = 0; t < MT; ++t) xr[t] = xh + (m0 + (t < nt ? t : 0)) * K;
         float acc[R][MT];
 #pragma unroll
         for (int i = 0; i < R; ++i)
 #pragma unroll
             for (int t = 0; t < MT; ++t) acc[i][t] = 0.0f;
 
-        for (int64_t c = lane; c < nchunk; c += 32) {
-            // activation chunk -> fp32
-            float xf[MT][CE];
+        if (warp_active) {
+            for (int64_t cb = c_begin; cb < c_end; cb += 32 * J) {
+                // issue every load of the batch first
+                uint4 wq[R][J];
+                uint16_t s2[R][J];
 #pragma unroll
-            for (int t = 0; t < MT; ++t) {
+                for (int j = 0; j < J; ++j) {
+                    const int64_t c = cb + lane + 32 * j;
+                    const bool ok = c < c_end;
 #pragma unroll
-                for (int q = 0; q < CE / 8; ++q) {
-                    uint4 v = ldg_v4(xr[t] + c * CE + q * 8);
-                    uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        xf[t][q * 8 + 2 * j] = bf16lo_to_f32(u[j]);
-                        xf[t][q * 8 + 2 * j + 1] = bf16hi_to_f32(u[j]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < R; ++i) {
-                uint32_t w[VB / 4];
-                load_codes<VB>(codes + wrow[i] * (K >> 1) + c * VB, w);
-                float sd[NB];
-                if constexpr (NB == 2) {
-                    const uint16_t s2 = __ldg(reinterpret_cast<const uint16_t*>(
-                        scales + sf_offset<LAYOUT>(wrow[i], 2 * c, nsf)));
-                    const float2 f = f16x2_to_f32x2(e4m3x2_to_f16x2(s2));
-                    sd[0] = f.x;
-                    sd[NB - 1] = f.y;
-                } else {
-                    sd[0] = e4m3_to_f32(__ldg(scales + sf_offset<LAYOUT>(wrow[i], c, nsf)));
-                }
-                float wf[CE];
-#pragma unroll
-                for (int j = 0; j < VB / 4; ++j) {
-                    uint32_t h[4];
-                    e2m1x8_to_f16x2(w[j], h);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float2 f = f16x2_to_f32x2(h[q]);
-                        wf[8 * j + 2 * q] = f.x;
-                        wf[8 * j + 2 * q + 1] = f.y;
+                    for (int i = 0; i < R; ++i) {
+                        if (ok) {
+                            wq[i][j] = ldg_stream(codes + wrow[i] * (K >> 1) + c * 16);
+                            s2[i][j] = __ldg(reinterpret_cast<const uint16_t*>(
+                                scales + sf_offset<LAYOUT>(wrow[i], 2 * c, nsf)));
+                        } else {
+                            wq[i][j] = make_uint4(0, 0, 0, 0);
+                            s2[i][j] = 0;
+                        }
                     }
                 }
 #pragma unroll
-                for (int t = 0; t < MT; ++t) {
+                for (int j = 0; j < J; ++j) {
+                    const int64_t c = cb + lane + 32 * j;
+                    if (c >= c_end) break;
 #pragma unroll
-                    for (int bb = 0; bb < NB; ++bb) {
-                        float p = 0.0f;
+                    for (int t = 0; t < MT; ++t) {
+                        uint32_t xw[16];
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) p = fmaf(xf[t][16 * bb + j], wf[16 * bb + j], p);
-                        acc[i][t] = fmaf(p, sd[bb], acc[i][t]);
+                        for (int v = 0; v < 4; ++v) {
+                            const uint4 xv = ldg_v4(xr[t] + c * 32 + v * 8);
+                            xw[4 * v] = xv.x; xw[4 * v + 1] = xv.y; xw[4 * v + 2] = xv.z; xw[4 * v + 3] = xv.w;
+                        }
+#pragma unroll
+                        for (int i = 0; i < R; ++i) {
+                            float p0 = 0.0f, p1 = 0.0f;
+                            chunk_dot(wq[i][j], xw, p0, p1);
+                            const float2 sd = f16x2_to_f32x2(e4m3x2_to_f16x2(s2[i][j]));
+                            acc[i][t] = fmaf(p0, sd.x, acc[i][t]);
+                            acc[i][t] = fmaf(p1, sd.y, acc[i][t]);
+                        }
                     }
                 }
             }
         }
-
 #pragma unroll
         for (int i = 0; i < R; ++i)
 #pragma unroll
             for (int t = 0; t < MT; ++t) acc[i][t] = warp_sum(acc[i][t]);
 
-        OutT* y = reinterpret_cast<OutT*>(a.y);
+        if constexpr (QS > 1) {
+            if (lane == 0) {
 #pragma unroll
-        for (int i = 0; i < RW; ++i) {
+                for (int i = 0; i < R; ++i)
 #pragma unroll
-            for (int t = 0; t < MT; ++t) {
-                if (lane == ((i * MT + t) & 31) && t < nt && cvalid[i]) {
-                    float v;
-                    if constexpr (EPI == NVFP4_EPI_SWIGLU) {
-                        const float g = acc[i][t] * gs, u = acc[RW + i][t] * gs;
-                        v = g / (1.0f + expf(-g)) * u;
-                    } else {
-                        v = acc[i][t] * gs;
+                    for (int t = 0; t < MT; ++t) red[warp][i][t] = acc[i][t];
+            }
+            __syncthreads();
+            if (q == 0) {
+#pragma unroll
+                for (int i = 0; i < R; ++i)
+#pragma unroll
+                    for (int t = 0; t < MT; ++t) {
+                        float s = 0.0f;
+#pragma unroll
+                        for (int qq = 0; qq < QS; ++qq) s += red[g * QS + qq][i][t];
+                        acc[i][t] = s;
                     }
-                    store_out<OutT>(y + (m0 + t) * a.ldy + col0 + i, v);
+            }
+            __syncthreads();
+        }
+
+        if (q == 0 && warp_active) {
+            OutT* y = reinterpret_cast<OutT*>(a.y);
+#pragma unroll
+            for (int i = 0; i < RW; ++i) {
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                    if (lane == ((i * MT + t) & 31) && t < nt && cvalid[i]) {
+                        const float sc = gs * a.inv_scale[m0 + t];
+                        float v;
+                        if constexpr (EPI == NVFP4_EPI_SWIGLU) {
+                            const float gg = acc[0][t] * sc, u = acc[1][t] * sc;
+                            v = gg / (1.0f + expf(-gg)) * u;
+                        } else {
+                            v = acc[i][t] * sc;
+                        }
+                        store_out<OutT>(y + (m0 + t) * a.ldy + col0 + i, v);
+                    }
                 }
             }
         }
     }
 }
 
-template <int MT, int R, int VB, int LAYOUT, typename OutT, int EPI>
+// ---- K % 32 == 16 tail path (8-byte rows): one warp per row, plain loads -----
+template <int LAYOUT, typename OutT>
+__global__ void __launch_bounds__(256) gemv_w4a16_odd_kernel(const GemvArgs a) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t n = (int64_t)blockIdx.y * 8 + warp;
+    if (n >= a.N) return;
+    const int64_t K = a.K, nsf = K >> 4;
+    const int64_t m = blockIdx.x;
+    const __half* xr = reinterpret_cast<const __half*>(a.xh) + m * K;
+    float acc = 0.0f;
+    for (int64_t b = lane; b < nsf; b += 32) {   // one 16-element block per step
+        uint2 wv;
+        asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                     : "=r"(wv.x), "=r"(wv.y) : "l"(a.codes + n * (K >> 1) + b * 8));
+        const uint4 xv0 = ldg_v4(xr + b * 16), xv1 = ldg_v4(xr + b * 16 + 8);
+        const uint32_t xw[8] = {xv0.x, xv0.y, xv0.z, xv0.w, xv1.x, xv1.y, xv1.z, xv1.w};
+        const uint32_t w[2] = {wv.x, wv.y};
+        float p = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            uint32_t h[4];
+            e2m1x8_to_f16x2(w[j], h);
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+                p = fma_f16((uint16_t)(h[qq] & 0xFFFF), (uint16_t)(xw[4 * j + qq] & 0xFFFF), p);
+                p = fma_f16((uint16_t)(h[qq] >> 16), (uint16_t)(xw[4 * j + qq] >> 16), p);
+            }
+        }
+        acc = fmaf(p, e4m3_to_f32(__ldg(a.scales + sf_offset<LAYOUT>(n, b, nsf))), acc);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) store_out<OutT>(reinterpret_cast<OutT*>(a.y) + m * a.ldy + n, acc * a.gs[0] * a.inv_scale[m]);
+}
+
+template <int MT, int R, int QS, int J, int LAYOUT, typename OutT, int EPI>
 static int launch_cfg(const GemvArgs& a, cudaStream_t st) {
-    constexpr int RW = (EPI == NVFP4_EPI_SWIGLU) ? R / 2 : R;
+    constexpr int RG = 8 / QS;
+    constexpr int RW = (EPI == NVFP4_EPI_SWIGLU) ? 1 : R;
     const int64_t ncols = (EPI == NVFP4_EPI_SWIGLU) ? a.N / 2 : a.N;
-    const int64_t tiles = (ncols + 8 * RW - 1) / (8 * RW);
+    const int64_t tiles = (ncols + RG * RW - 1) / (RG * RW);
     const int64_t gx = a.offsets ? a.E : (a.M + MT - 1) / MT;
     if (tiles > 65535 || gx > 0x7fffffff) return NVFP4_ERR_SHAPE;
     dim3 grid((unsigned)gx, (unsigned)tiles);
-    gemv_w4a16_kernel<MT, R, VB, LAYOUT, OutT, EPI><<<grid, 256, 0, st>>>(a);
+    gemv_w4a16_kernel<MT, R, QS, J, LAYOUT, OutT, EPI><<<grid, 256, 0, st>>>(a);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 
-template <int VB, int LAYOUT, typename OutT, int EPI>
-static int launch_mt(const GemvArgs& a, int64_t rows_hint, cudaStream_t st) {
-    if (rows_hint <= 1) return launch_cfg<1, 4, VB, LAYOUT, OutT, EPI>(a, st);
-    if (rows_hint <= 2) return launch_cfg<2, 2, VB, LAYOUT, OutT, EPI>(a, st);
-    return launch_cfg<4, 2, VB, LAYOUT, OutT, EPI>(a, st);
+// K-split per CTA: enough CTAs for 148 SMs when N is small, 1 when N is large.
+template <int MT, int LAYOUT, typename OutT, int EPI>
+static int launch_qs(const GemvArgs& a, cudaStream_t st) {
+    const int64_t ncols = (EPI == NVFP4_EPI_SWIGLU) ? a.N / 2 : a.N;
+    const int64_t rows_per_warp = (EPI == NVFP4_EPI_SWIGLU) ? 1 : 2;
+    const int64_t warps_at_qs1 = (ncols + rows_per_warp - 1) / rows_per_warp * (a.offsets ? 1 : (a.M + MT - 1) / MT);
+    const int64_t nch = a.K >> 5;
+    // target: >= ~8 resident-warp-slots of work per SM (148 SMs x 32 warps)
+    int qs = 1;
+    while (qs < 8 && warps_at_qs1 * qs < 148 * 48 && nch / (qs * 2) >= 16) qs *= 2;
+    if (a.offsets) qs = nch >= 128 ? 2 : 1;
+    switch (qs) {
+        case 1: return launch_cfg<MT, 2, 1, 6, LAYOUT, OutT, EPI>(a, st);
+        case 2: return launch_cfg<MT, 2, 2, 6, LAYOUT, OutT, EPI>(a, st);
+        case 4: return launch_cfg<MT, 2, 4, 5, LAYOUT, OutT, EPI>(a, st);
+        default: return launch_cfg<MT, 2, 8, 3, LAYOUT, OutT, EPI>(a, st);
+    }
 }
 
-template <int VB, int LAYOUT>
-static int launch_out(const GemvArgs& a, int64_t rows_hint, cudaStream_t st) {
-    if (a.epilogue == NVFP4_EPI_SWIGLU) {
-        if (a.y_dtype == NVFP4_DTYPE_BF16) return launch_mt<VB, LAYOUT, __nv_bfloat16, NVFP4_EPI_SWIGLU>(a, rows_hint, st);
-        return launch_mt<VB, LAYOUT, float, NVFP4_EPI_SWIGLU>(a, rows_hint, st);
+template <int LAYOUT, typename OutT, int EPI>
+static int launch_mt(const GemvArgs& a, cudaStream_t st) {
+    const int64_t rows_hint = a.offsets ? 4 : a.M;
+    if (rows_hint <= 1) return launch_qs<1, LAYOUT, OutT, EPI>(a, st);
+    if (rows_hint <= 2) return launch_qs<2, LAYOUT, OutT, EPI>(a, st);
+    return launch_qs<4, LAYOUT, OutT, EPI>(a, st);
+}
+
+template <int LAYOUT>
+static int launch_layout(const GemvArgs& a, cudaStream_t st) {
+    if (a.K % 32) {
+        if (a.offsets || a.epilogue != NVFP4_EPI_NONE) return NVFP4_ERR_SHAPE;
+        dim3 grid((unsigned)a.M, (unsigned)((a.N + 7) / 8));
+        if (a.y_dtype == NVFP4_DTYPE_BF16)
+            gemv_w4a16_odd_kernel<LAYOUT, __nv_bfloat16><<<grid, 256, 0, st>>>(a);
+        else
+            gemv_w4a16_odd_kernel<LAYOUT, float><<<grid, 256, 0, st>>>(a);
+        return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
     }
-    if (a.y_dtype == NVFP4_DTYPE_BF16) return launch_mt<VB, LAYOUT, __nv_bfloat16, NVFP4_EPI_NONE>(a, rows_hint, st);
-    return launch_mt<VB, LAYOUT, float, NVFP4_EPI_NONE>(a, rows_hint, st);
+    if (a.epilogue == NVFP4_EPI_SWIGLU) {
+        if (a.y_dtype == NVFP4_DTYPE_BF16) return launch_mt<LAYOUT, __nv_bfloat16, NVFP4_EPI_SWIGLU>(a, st);
+        return launch_mt<LAYOUT, float, NVFP4_EPI_SWIGLU>(a, st);
+    }
+    if (a.y_dtype == NVFP4_DTYPE_BF16) return launch_mt<LAYOUT, __nv_bfloat16, NVFP4_EPI_NONE>(a, st);
+    return launch_mt<LAYOUT, float, NVFP4_EPI_NONE>(a, st);
+}
+
+int launch_x_prep(const void* x, const int32_t* gather, int64_t rows, int64_t K, void* xh, float* inv_scale,
+                  cudaStream_t st) {
+    if (rows > 0x7fffffff) return NVFP4_ERR_SHAPE;
+    x_prep_kernel<<<(unsigned)rows, 256, 0, st>>>((const __nv_bfloat16*)x, gather, K, (__half*)xh, inv_scale);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 
 int launch_gemv_w4a16(const GemvArgs& a, cudaStream_t st) {
-    // Dense: token-group width from M.  Grouped: rows per expert vary; the
-    // widest group (4) amortises the weight read for hot experts.
-    const int64_t rows_hint = a.offsets ? 4 : a.M;
-    const bool v16 = (a.K % 32) == 0;
-    if (a.sf_layout == NVFP4_SF_TILED)
-        return v16 ? launch_out<16, NVFP4_SF_TILED>(a, rows_hint, st) : launch_out<8, NVFP4_SF_TILED>(a, rows_hint, st);
-    return v16 ? launch_out<16, NVFP4_SF_ROWMAJOR>(a, rows_hint, st)
-               : launch_out<8, NVFP4_SF_ROWMAJOR>(a, rows_hint, st);
+    if (a.sf_layout == NVFP4_SF_TILED) return launch_layout<NVFP4_SF_TILED>(a, st);
+    return launch_layout<NVFP4_SF_ROWMAJOR>(a, st);
 }
 
 }  // namespace nvfp4

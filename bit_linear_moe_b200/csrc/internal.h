@@ -15,8 +15,8 @@ int launch_quantize(const void* x, int x_dtype, const int32_t* src_rows, int64_t
 
 // gemv.cu: W4A16 on CUDA cores.
 struct GemvArgs {
-    const void* x;            // bf16 activations, row stride K
-    const int32_t* gather;    // grouped: activation row of output row r is gather[r] (nullable)
+    const void* xh;           // fp16 activations x * 2^p (from launch_x_prep), [rows, K]
+    const float* inv_scale;   // per activation row: 2^-p
     int64_t M;                // dense: number of rows of x / y
     int64_t K;
     const uint8_t* codes;     // [N, K/2]  (grouped: [E, N, K/2])
@@ -32,7 +32,16 @@ struct GemvArgs {
     int y_dtype;              // NVFP4_DTYPE_F32 / BF16
     int64_t ldy;              // elements per output row
 };
+// Activation prep for W4A16: xh[r] = fp16(x[src(r)] * 2^p_r), inv_scale[r] = 2^-p_r,
+// src(r) = gather[r] if gather else r.
+int launch_x_prep(const void* x, const int32_t* gather, int64_t rows, int64_t K, void* xh, float* inv_scale,
+                  cudaStream_t st);
 int launch_gemv_w4a16(const GemvArgs& a, cudaStream_t st);
+
+// gemv_tma.cu: pipelined W4A16 decode (TMA ring, cluster split-K) for M <= 4, K % 256 == 0.
+bool decode_tma_supported(int64_t M, int64_t K, int64_t N);
+int launch_decode_tma(const void* x, int64_t M, int64_t K, const uint8_t* codes, const uint8_t* scales,
+                      int sf_layout, const float* gs, int64_t N, void* y, int y_dtype, int* status, cudaStream_t st);
 
 // moe.cu
 int launch_router_logits(const void* h, const void* wr, const float* bias, int64_t T, int64_t H, int32_t E,

@@ -75,8 +75,14 @@ def test_linear_validation(L):
     assert _linear(L, yd=7) == nv.ERR_DTYPE
     assert _linear(L, lay=5) == nv.ERR_LAYOUT
     assert _linear(L, mode=9) == nv.ERR_MODE
+    need = L.nvfp4_linear_workspace(1, 64, 16, nv.MODE_W4A16)
+    assert need >= 64 * 2 + 4
+    assert _linear(L) == nv.ERR_WORKSPACE
+    assert _linear(L, ws=FAKE2, wsb=need - 1) == nv.ERR_WORKSPACE
+    assert _linear(L, ws=MISALIGNED, wsb=need) == nv.ERR_ALIGN
+    assert _linear(L, N=200000, ws=FAKE2, wsb=need) == nv.ERR_SHAPE
     if not torch.cuda.is_available():
-        assert _linear(L) == nv.ERR_ARCH
+        assert _linear(L, ws=FAKE2, wsb=need) == nv.ERR_ARCH
 
 
 def test_linear_w4a4_validation(L):
@@ -141,5 +147,6 @@ def test_grouped_validation(L):
     assert g(epi=nv.EPI_COMBINE, tw=FAKE, ro=FAKE, k=3) == nv.ERR_SHAPE
     assert g(epi=nv.EPI_SWIGLU, N=33) == nv.ERR_SHAPE
     assert g(epi=7) == nv.ERR_MODE
+    assert g(K=48) == nv.ERR_SHAPE
     if not torch.cuda.is_available():
         assert g() == nv.ERR_ARCH
