@@ -167,6 +167,7 @@ int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t
     if (mode == NVFP4_MODE_W4A4) {
         if (w_sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_LAYOUT;
         if (K % 256) return NVFP4_ERR_SHAPE;
+        if ((N + 127) / 128 > 65535) return NVFP4_ERR_SHAPE;
     } else if (N > kMaxW4A16N || M > kMaxW4A16M) {
         return NVFP4_ERR_SHAPE;
     }
@@ -174,8 +175,18 @@ int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t
     if (need && (!ws || ws_bytes < need)) return NVFP4_ERR_WORKSPACE;
     if (need && !aligned16(ws)) return NVFP4_ERR_ALIGN;
     NVFP4_TRY(check_arch());
-    if (mode == NVFP4_MODE_W4A4) return NVFP4_ERR_MODE;  // tensor-core path not wired yet
     cudaStream_t st = (cudaStream_t)stream;
+    if (mode == NVFP4_MODE_W4A4) {
+        // activations -> NVFP4 (per-tensor gs, tiled scales) in the workspace, then the tensor-core GEMM
+        char* wp = (char*)ws;
+        unsigned* amax = (unsigned*)wp;
+        float* gs_x = (float*)(wp + 16);
+        uint8_t* xc = (uint8_t*)(wp + 256);
+        uint8_t* xs = xc + align256((size_t)(M * K / 2));
+        NVFP4_TRY(launch_amax(x, NVFP4_DTYPE_BF16, M * K, amax, st));
+        NVFP4_TRY(launch_quantize(x, NVFP4_DTYPE_BF16, nullptr, M, K, NVFP4_SF_TILED, nullptr, amax, xc, xs, gs_x, st));
+        return launch_gemm_w4a4(xc, xs, gs_x, M, K, w_codes, w_scales, w_gs, N, y, y_dtype, device_status_ptr(), st);
+    }
     if (decode_tma_supported(M, K, N))
         return launch_decode_tma(x, M, K, w_codes, w_scales, w_sf_layout, w_gs, N, y, y_dtype, device_status_ptr(),
                                  st);
@@ -289,8 +300,8 @@ int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const 
     if (need && (!ws || ws_bytes < need)) return NVFP4_ERR_WORKSPACE;
     if (need && !aligned16(ws)) return NVFP4_ERR_ALIGN;
     NVFP4_TRY(check_arch());
-    if (mode == NVFP4_MODE_W4A4) return NVFP4_ERR_MODE;  // tensor-core path not wired yet
     cudaStream_t st = (cudaStream_t)stream;
+    if (mode == NVFP4_MODE_W4A4) return NVFP4_ERR_MODE;  // grouped tensor-core path not wired yet
     char* wp = (char*)ws;
     float* d = nullptr;
     if (epilogue == NVFP4_EPI_COMBINE) {

@@ -43,6 +43,12 @@ bool decode_tma_supported(int64_t M, int64_t K, int64_t N);
 int launch_decode_tma(const void* x, int64_t M, int64_t K, const uint8_t* codes, const uint8_t* scales,
                       int sf_layout, const float* gs, int64_t N, void* y, int y_dtype, int* status, cudaStream_t st);
 
+// gemm_w4a4.cu: tcgen05 block-scaled W4A4 GEMM.  A = activations [M, K/2]
+// codes + TILED scales, B = weights [N, K/2] + TILED scales; K % 256 == 0.
+int launch_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales, const float* gs_a, int64_t M, int64_t K,
+                     const uint8_t* b_codes, const uint8_t* b_scales, const float* gs_b, int64_t N, void* y,
+                     int y_dtype, int* status, cudaStream_t st);
+
 // moe.cu
 int launch_router_logits(const void* h, const void* wr, const float* bias, int64_t T, int64_t H, int32_t E,
                          float* logits, cudaStream_t st);
