@@ -272,6 +272,7 @@ def run_native(args, rank, world, dist):
     extra = {"decode_m1_per_shape": per_shape}
     if not args.quick:
         extra["decode_sweep"] = decode_sweep(nv, torch, dev, layers)
+        extra["prefill"] = prefill_section(nv, torch, dev, layers)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -333,6 +334,74 @@ def decode_sweep(nv, torch, dev, layers, reps=200):
             m = a.elapsed_time(b) / reps
             row[str(M)] = round(decode_bytes(M, K, N) / (m * 1e-3) / 1e9, 1)
         out[name] = row
+    return out
+
+
+def _time_graphs(torch, graphs, reps):
+    stream = torch.cuda.current_stream()
+    for i in range(3):
+        graphs[i % len(graphs)].replay()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(reps):
+        graphs[i % len(graphs)].replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def _capture(torch, dev, fn_per_copy):
+    stream = torch.cuda.current_stream()
+    side = torch.cuda.Stream(device=dev)
+    for i in range(2):
+        fn_per_copy(i)
+    torch.cuda.synchronize()
+    side.wait_stream(stream)
+    graphs = []
+    with torch.cuda.stream(side):
+        for i in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                fn_per_copy(i)
+            graphs.append(g)
+    stream.wait_stream(side)
+    return graphs
+
+
+def prefill_section(nv, torch, dev, layers, M=2048, reps=30):
+    """W4A4 prefill at M tokens on the four shapes: TFLOP/s = 2 M N K / time,
+    GEMM alone (pre-quantized activations) and with the activation quantize."""
+    from bit_linear_moe_b200 import synth
+    seeds = dict((s[0], s[3]) for s in SHAPES)
+    out = {"M": M, "shapes": {}}
+    tot_flop = tot_gemm = tot_e2e = 0.0
+    for name, K, N, copies, _, _ in layers:
+        x = torch.from_numpy(synth.prefill_x(seeds[name], M, K)[0]).to(torch.bfloat16).to(dev)
+        xc, xs, xg = nv.nvfp4_quantize(x, sf_layout=nv.SF_TILED)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(int(nv.lib().nvfp4_linear_workspace(M, K, N, nv.MODE_W4A4)), dtype=torch.uint8, device=dev)
+
+        def gemm(i):
+            c, s, g = copies[i]
+            nv.nvfp4_linear_w4a4q(xc, xs, xg, c, s, g, y=y)
+
+        def e2e(i):
+            c, s, g = copies[i]
+            nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A4, ws=ws)
+
+        t_g = _time_graphs(torch, _capture(torch, dev, gemm), reps)
+        t_e = _time_graphs(torch, _capture(torch, dev, e2e), reps)
+        flop = 2.0 * M * N * K
+        out["shapes"][name] = {"gemm_us": round(t_g * 1e3, 1), "gemm_TFLOPs": round(flop / (t_g * 1e-3) / 1e12, 1),
+                               "with_quant_us": round(t_e * 1e3, 1),
+                               "with_quant_TFLOPs": round(flop / (t_e * 1e-3) / 1e12, 1)}
+        tot_flop += flop
+        tot_gemm += t_g
+        tot_e2e += t_e
+    out["gemm_TFLOPs"] = round(tot_flop / (tot_gemm * 1e-3) / 1e12, 1)
+    out["with_quant_TFLOPs"] = round(tot_flop / (tot_e2e * 1e-3) / 1e12, 1)
+    out["peak_nominal_dense_nvfp4_TFLOPs"] = 9000.0
+    out["frac_of_nominal"] = round(out["gemm_TFLOPs"] / 9000.0, 4)
     return out
 
 

@@ -55,6 +55,7 @@ def lib() -> ctypes.CDLL:
             "nvfp4_quantize": (i, [p, i, i64, i64, p, i, p, p, p, p, sz, p]),
             "nvfp4_linear_workspace": (sz, [i64, i64, i64, i]),
             "nvfp4_linear": (i, [p, i, i64, i64, p, p, i, p, i64, p, i, i, p, sz, p]),
+            "nvfp4_linear_w4a4q": (i, [p, p, p, i64, i64, p, p, p, i64, p, i, p]),
             "moe_route_topk_workspace": (sz, [i64, i32, i32]),
             "moe_route_topk": (i, [p, p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p, sz, p]),
             "moe_grouped_linear_workspace": (sz, [i64, i64, i64, i32, i32, i, i]),
@@ -134,6 +135,18 @@ def nvfp4_linear(x: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor,
     _check(lib().nvfp4_linear(_ptr(x), _dtype_code(x), M, K, _ptr(w_codes), _ptr(w_scales), w_sf_layout,
                               _ptr(w_gs), N, _ptr(y), _dtype_code(y), mode, _ptr(ws), wsb, _stream()),
            "nvfp4_linear")
+    return y
+
+
+def nvfp4_linear_w4a4q(x_codes: torch.Tensor, x_scales: torch.Tensor, x_gs: torch.Tensor, w_codes: torch.Tensor,
+                       w_scales: torch.Tensor, w_gs: torch.Tensor, y=None, y_dtype=torch.bfloat16):
+    """W4A4 with pre-quantized activations (codes [M, K/2], TILED scales, device gs)."""
+    M, K = x_codes.shape[0], x_codes.shape[1] * 2
+    N = w_codes.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=x_codes.device)
+    _check(lib().nvfp4_linear_w4a4q(_ptr(x_codes), _ptr(x_scales), _ptr(x_gs), M, K, _ptr(w_codes), _ptr(w_scales),
+                                    _ptr(w_gs), N, _ptr(y), _dtype_code(y), _stream()), "nvfp4_linear_w4a4q")
     return y
 
 

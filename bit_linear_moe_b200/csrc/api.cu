@@ -211,6 +211,21 @@ int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t
     return launch_gemv_w4a16(a, st);
 }
 
+int nvfp4_linear_w4a4q(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_gs, int64_t M, int64_t K,
+                       const uint8_t* w_codes, const uint8_t* w_scales, const float* w_gs, int64_t N, void* y,
+                       int y_dtype, void* stream) {
+    if (!x_codes || !x_scales || !x_gs || !w_codes || !w_scales || !w_gs || !y) return NVFP4_ERR_NULL;
+    if (!dtype_ok(y_dtype)) return NVFP4_ERR_DTYPE;
+    if (M < 1 || N < 1 || K < 256 || K % 256 || M > ((int64_t)1 << 31) || (N + 127) / 128 > 65535 ||
+        K > ((int64_t)1 << 24))
+        return NVFP4_ERR_SHAPE;
+    if (!aligned16(x_codes) || !aligned16(x_scales) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y))
+        return NVFP4_ERR_ALIGN;
+    NVFP4_TRY(check_arch());
+    return launch_gemm_w4a4(x_codes, x_scales, x_gs, M, K, w_codes, w_scales, w_gs, N, y, y_dtype,
+                            device_status_ptr(), (cudaStream_t)stream);
+}
+
 // ---- MoE routing -------------------------------------------------------------------
 
 static int64_t perm_blocks(int64_t T) { return (T + kPermBlockTokens - 1) / kPermBlockTokens; }

@@ -157,6 +157,20 @@ int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K,
                  void* y, int y_dtype, int mode,
                  void* ws, size_t ws_bytes, void* stream);
 
+/* ---- nvfp4_linear_w4a4q ---------------------------------------------------
+ * The W4A4 linear with activations already in NVFP4 (e.g. written by a
+ * previous layer's quantizing epilogue, or by nvfp4_quantize with
+ * sf_layout = TILED): the tensor-core GEMM alone, without the quantize pass
+ * (Ignis README, "Credits": the NVFP4-full target).
+ *     y[m, n] = (*x_gs) * (*w_gs) * sum_k E2M1(xc) E4M3(xs) E2M1(wc) E4M3(ws)
+ *   x_codes  [M, K/2];  x_scales TILED for M rows;  x_gs one device float
+ *   w_codes  [N, K/2];  w_scales TILED for N rows;  w_gs one device float
+ *   y        [M, N] in y_dtype (F32 or BF16)
+ * Requires K % 256 == 0; no workspace. */
+int nvfp4_linear_w4a4q(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_gs, int64_t M, int64_t K,
+                       const uint8_t* w_codes, const uint8_t* w_scales, const float* w_gs, int64_t N,
+                       void* y, int y_dtype, void* stream);
+
 /* ---- moe_route_topk ------------------------------------------------------
  * Router of a routed mixture-of-experts layer (CHImp Alpha v1.0 model card,
  * "How it fits on one GPU": 10 of 512 experts per token).
