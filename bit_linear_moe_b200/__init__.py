@@ -58,6 +58,7 @@ def lib() -> ctypes.CDLL:
             "nvfp4_linear_w4a4q": (i, [p, p, p, i64, i64, p, p, p, i64, p, i, p]),
             "moe_route_topk_workspace": (sz, [i64, i32, i32]),
             "moe_route_topk": (i, [p, p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p, sz, p]),
+            "moe_route_topk_noalloc": (i, [p, p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p]),
             "moe_grouped_linear_workspace": (sz, [i64, i64, i64, i32, i32, i, i]),
             "moe_grouped_linear": (i, [p, i, i64, i, p, p, i32, i64, p, p, i, p, i64, i, p, p, i32, p, i, i,
                                        p, sz, p]),
@@ -171,6 +172,30 @@ def moe_route_topk(h: torch.Tensor, w_router: torch.Tensor, k: int, logit_bias=N
                                 _ptr(o["topk_idx"]), _ptr(o["topk_w"]), _ptr(o["expert_offsets"]),
                                 _ptr(o["perm_tok"]), _ptr(o["perm_slot"]), _ptr(o["row_of"]), _ptr(ws), wsb,
                                 _stream()), "moe_route_topk")
+    return o
+
+
+def moe_route_topk_noalloc(h: torch.Tensor, w_router: torch.Tensor, k: int, logit_bias=None,
+                           want_logits: bool = False, out=None):
+    """``moe_route_topk`` without a workspace: for callers that cannot allocate
+    device memory while routing.  The library's built-in 1 MiB scratch is used
+    instead (shared by every call; overlapping calls race)."""
+    T, H = h.shape
+    E = w_router.shape[0]
+    dev = h.device
+    o = dict(out or {})
+    if want_logits and "logits" not in o:
+        o["logits"] = torch.empty((T, E), dtype=torch.float32, device=dev)
+    o.setdefault("topk_idx", torch.empty((T, k), dtype=torch.int32, device=dev))
+    o.setdefault("topk_w", torch.empty((T, k), dtype=torch.float32, device=dev))
+    o.setdefault("expert_offsets", torch.empty(E + 1, dtype=torch.int32, device=dev))
+    o.setdefault("perm_tok", torch.empty(T * k, dtype=torch.int32, device=dev))
+    o.setdefault("perm_slot", torch.empty(T * k, dtype=torch.int32, device=dev))
+    o.setdefault("row_of", torch.empty((T, k), dtype=torch.int32, device=dev))
+    _check(lib().moe_route_topk_noalloc(_ptr(h), _ptr(w_router), _ptr(logit_bias), T, H, E, k,
+                                        _ptr(o.get("logits")), _ptr(o["topk_idx"]), _ptr(o["topk_w"]),
+                                        _ptr(o["expert_offsets"]), _ptr(o["perm_tok"]), _ptr(o["perm_slot"]),
+                                        _ptr(o["row_of"]), _stream()), "moe_route_topk_noalloc")
     return o
 
 

@@ -196,6 +196,27 @@ int moe_route_topk(const void* h, const void* w_router, const float* logit_bias,
                    int32_t* expert_offsets, int32_t* perm_tok, int32_t* perm_slot,
                    int32_t* row_of, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- moe_route_topk_noalloc ------------------------------------------------
+ * The pages have no counterpart to this call.  It computes exactly what
+ * moe_route_topk computes, for callers that cannot allocate device memory
+ * when they route (an engine whose device memory plan is fixed at load and
+ * must not grow inside a step, or code where an allocation would stall the
+ * device or is not permitted), so it takes no workspace.  Its scratch is a
+ * 1 MiB array inside the library that every GPU loading the library holds
+ * until exit.  It needs ceil(T/128) * E * 8 bytes (rounded up to 256-byte
+ * pieces), plus T * E * 4 bytes when logits_out is NULL; a request that does
+ * not fit returns NVFP4_ERR_WORKSPACE before launching anything (pass
+ * logits_out to route large T).  The first call on a device looks up the
+ * array's device address, so make it before any stream capture.  Every call
+ * shares the array: calls that overlap on the GPU race and must be
+ * serialized by the caller.  Arguments, layouts and errors are otherwise
+ * those of moe_route_topk. */
+int moe_route_topk_noalloc(const void* h, const void* w_router, const float* logit_bias,
+                           int64_t T, int64_t H, int32_t E, int32_t k,
+                           float* logits_out, int32_t* topk_idx, float* topk_w,
+                           int32_t* expert_offsets, int32_t* perm_tok, int32_t* perm_slot,
+                           int32_t* row_of, void* stream);
+
 /* ---- moe_grouped_linear --------------------------------------------------
  * Expert linears over the permuted rows (CHImp, same section: only the chosen
  * experts' weights are read).  For each expert e and row r in
