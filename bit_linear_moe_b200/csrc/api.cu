@@ -61,8 +61,45 @@ constexpr int64_t kMaxW4A16M = (int64_t)1 << 30;
 // W4A16 workspace: fp16 activations and one inverse scale per row.
 static size_t w4a16_ws(int64_t rows, int64_t K) { return align256((size_t)(rows * K) * 2) + align256((size_t)rows * 4); }
 
-// Row padding of a W4A4 operand: the tensor-core tiles are 128 rows.
-static int64_t moe_w4a4_rows(int64_t R, int32_t E) { return R + (int64_t)E * 127; }
+// Padded rows of the grouped W4A4 operand: every expert's rows padded to whole
+// 128-row tiles (at most 127 padding rows per expert), rounded up to a tile.
+static int64_t moe_w4a4_rows(int64_t R, int32_t E) { return (R + (int64_t)E * 127 + 127) / 128 * 128; }
+
+struct GroupedW4A4Ws {
+    unsigned* amax;
+    float* gs_x;
+    int32_t* pad_off;
+    int32_t* tile_info;
+    int32_t* src_rows;
+    uint8_t* codes;
+    uint8_t* scales;
+    float* yacc;
+    int32_t* tok_of;
+    float* w_of;
+    size_t bytes;
+};
+static GroupedW4A4Ws grouped_w4a4_ws(void* base, int64_t R, int64_t K, int64_t N, int32_t E, int32_t k,
+                                     int epilogue) {
+    GroupedW4A4Ws w{};
+    const int64_t rp = moe_w4a4_rows(R, E);
+    char* p = (char*)base;
+    size_t off = 0;
+    auto take = [&](size_t n) { char* q = p ? p + off : nullptr; off += align256(n); return q; };
+    w.amax = (unsigned*)take(16);
+    w.gs_x = (float*)take(16);
+    w.pad_off = (int32_t*)take((size_t)(E + 1) * 4);
+    w.tile_info = (int32_t*)take((size_t)(rp / 128) * 12);
+    w.src_rows = (int32_t*)take((size_t)rp * 4);
+    w.codes = (uint8_t*)take((size_t)(rp * K / 2));
+    w.scales = (uint8_t*)take(scales_bytes(rp, K, NVFP4_SF_TILED));
+    if (epilogue == NVFP4_EPI_COMBINE && k > 0) {
+        w.yacc = (float*)take((size_t)(R / k) * (size_t)N * 4);
+        w.tok_of = (int32_t*)take((size_t)R * 4);
+        w.w_of = (float*)take((size_t)R * 4);
+    }
+    w.bytes = off;
+    return w;
+}
 }  // namespace nvfp4
 
 using namespace nvfp4;
@@ -273,13 +310,11 @@ size_t moe_grouped_linear_workspace(int64_t R, int64_t K, int64_t N, int32_t E, 
     (void)k;
     mode = resolve_grouped_mode(mode, R);
     size_t need = 0;
-    if (epilogue == NVFP4_EPI_COMBINE) need += align256((size_t)(R * N) * 4);
-    if (mode == NVFP4_MODE_W4A16) need += w4a16_ws(R, K);
-    if (mode == NVFP4_MODE_W4A4) {
-        const int64_t rp = moe_w4a4_rows(R, E);
-        need += align256(256) + align256((size_t)(rp * K / 2)) + align256(scales_bytes(rp, K, NVFP4_SF_TILED)) +
-                align256((size_t)rp * 4);
+    if (mode == NVFP4_MODE_W4A16) {
+        if (epilogue == NVFP4_EPI_COMBINE) need += align256((size_t)(R * N) * 4);
+        need += w4a16_ws(R, K);
     }
+    if (mode == NVFP4_MODE_W4A4) need += grouped_w4a4_ws(nullptr, R, K, N, E, k, epilogue).bytes;
     return need;
 }
 
@@ -307,7 +342,9 @@ int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const 
     mode = resolve_grouped_mode(mode, R);
     if (mode == NVFP4_MODE_W4A4) {
         if (w_sf_layout != NVFP4_SF_TILED) return NVFP4_ERR_LAYOUT;
-        if (K % 256) return NVFP4_ERR_SHAPE;
+        if (K % 256 || N % 128 || (epilogue == NVFP4_EPI_SWIGLU && N % 256) || (int64_t)E * N > 0x7fffffff ||
+            moe_w4a4_rows(R, E) / 128 > 0x7fffffff)
+            return NVFP4_ERR_SHAPE;
     } else if (K % 32 || N > kMaxW4A16N) {
         return NVFP4_ERR_SHAPE;
     }
@@ -316,7 +353,30 @@ int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const 
     if (need && !aligned16(ws)) return NVFP4_ERR_ALIGN;
     NVFP4_TRY(check_arch());
     cudaStream_t st = (cudaStream_t)stream;
-    if (mode == NVFP4_MODE_W4A4) return NVFP4_ERR_MODE;  // grouped tensor-core path not wired yet
+    if (mode == NVFP4_MODE_W4A4) {
+        const int64_t rp = moe_w4a4_rows(R, E);
+        GroupedW4A4Ws w = grouped_w4a4_ws(ws, R, K, N, E, k, epilogue);
+        NVFP4_TRY(launch_moe_pad(expert_offsets, E, rp, gather ? perm_tok : nullptr, w.pad_off, w.tile_info,
+                                 w.src_rows, st));
+        NVFP4_TRY(launch_amax_rows(x, w.src_rows, rp, K, w.amax, st));
+        NVFP4_TRY(launch_quantize(x, NVFP4_DTYPE_BF16, w.src_rows, rp, K, NVFP4_SF_TILED, nullptr, w.amax, w.codes,
+                                  w.scales, w.gs_x, st, w.pad_off + E));
+        const int64_t sf_stride = (int64_t)scales_bytes(N, K, NVFP4_SF_TILED);
+        if (epilogue == NVFP4_EPI_COMBINE) {
+            const int64_t T = R / k;
+            float* acc = y_dtype == NVFP4_DTYPE_F32 ? (float*)y : w.yacc;
+            if (cudaMemsetAsync(acc, 0, (size_t)(T * N) * 4, st) != cudaSuccess) return NVFP4_ERR_LAUNCH;
+            NVFP4_TRY(launch_row_token(row_of, topk_w, R, k, w.tok_of, w.w_of, st));
+            NVFP4_TRY(launch_gemm_w4a4_grouped(w.codes, w.scales, w.gs_x, rp, K, w.tile_info, w_codes, w_scales,
+                                               sf_stride, w_gs, E, N, epilogue, nullptr, NVFP4_DTYPE_F32, acc,
+                                               w.tok_of, w.w_of, device_status_ptr(), st));
+            if (y_dtype == NVFP4_DTYPE_BF16) return launch_f32_to_bf16(acc, T * N, y, st);
+            return NVFP4_OK;
+        }
+        return launch_gemm_w4a4_grouped(w.codes, w.scales, w.gs_x, rp, K, w.tile_info, w_codes, w_scales, sf_stride,
+                                        w_gs, E, N, epilogue, y, y_dtype, nullptr, nullptr, nullptr,
+                                        device_status_ptr(), st);
+    }
     char* wp = (char*)ws;
     float* d = nullptr;
     if (epilogue == NVFP4_EPI_COMBINE) {

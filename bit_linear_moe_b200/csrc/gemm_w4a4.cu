@@ -1,4 +1,5 @@
-// K4: W4A4 linear on tcgen05 block-scaled tensor cores (kind::mxf4nvf4).
+// K4 / K7: W4A4 linear on tcgen05 block-scaled tensor cores (kind::mxf4nvf4),
+// dense and grouped by expert.
 //
 // Prefill runs in 2,048-token chunks on FP4 tensor cores (Ignis README,
 // "How fast"; "Credits": split-K prefill, the NVFP4-full target).  With both
@@ -10,19 +11,28 @@
 // scales of both operands and accumulates in fp32 in tensor memory; the two
 // per-tensor scales are applied in the epilogue.
 //
-// CTA (6 warps) computes one 128 x 128 output tile:
+// CTA (6 warps) computes one 128-row tile against one (or, for SwiGLU, two)
+// 128-row weight tiles:
 //   warp 0   allocates tensor memory; lane 0 streams, per 256-element K tile,
-//            A (128 x 128 B) and B (128 x 128 B) with 2D TMA (128-byte
-//            swizzle, no multicast) and their scale factors (two 2 KB runs of
-//            512-byte atoms, bulk copies) into a 3-stage ring;
-//   warp 1   lane 0 copies the scale atoms to tensor memory (tcgen05.cp,
-//            32x128b.warpx4) and issues 4 MMAs of K = 64 per stage, then
-//            commits to the stage's empty barrier;
-//   warps 2-5 wait for the last commit, read the 128 x 128 fp32 accumulator
-//            with tcgen05.ld (each warp its 32-lane quadrant), scale by
-//            gs_x * gs_w and store.
-// Two CTAs fit on an SM (108 KB of shared memory, 256 tensor-memory columns
-// each), so one CTA's epilogue overlaps the other's main loop.
+//            A and B (128 x 128 B each, 2D TMA with 128-byte swizzle, no
+//            multicast) and their scale factors (2 KB runs of 512-byte atoms,
+//            bulk copies) into a 3-stage ring;
+//   warp 1   lane 0 copies the scale atoms to tensor memory (tcgen05.cp
+//            32x128b.warpx4) and issues 4 MMAs of K = 64 per B tile and stage,
+//            then commits to the stage's empty barrier;
+//   warps 2-5 wait for the last commit, read the fp32 accumulators with
+//            tcgen05.ld (each warp its 32-lane quadrant) and run the epilogue.
+//
+// Grouped form (mixture of experts; CHImp Alpha v1.0 model card, "How it fits
+// on one GPU"): the permuted activations are laid out with each expert's rows
+// padded to whole 128-row tiles, and a tile table gives each 128-row tile its
+// expert, its first output row and its number of real rows; tiles past the
+// last expert exit at once.  The weight tile comes from the expert's rows of
+// the stacked [E * N, K/2] codes and the expert's scale block and gs.
+// Epilogues: NONE (y = acc * g); SWIGLU (gate tile = rows j0.. of the expert,
+// up tile = rows N/2 + j0..: two N = 128 MMAs into two accumulators, then
+// y = silu(g) * u); COMBINE (y[token] += topk_w * acc with fp32 vector
+// reductions; y is zeroed first).
 #include <cuda.h>
 
 #include <mutex>
@@ -33,45 +43,80 @@
 namespace nvfp4 {
 
 namespace w4a4 {
-constexpr int BM = 128, BN = 128, BK = 256;   // BK elements = 128 bytes per row
+constexpr int BM = 128, BN = 128, BK = 256;  // BK elements = 128 bytes per row
 constexpr int kStages = 3;
-constexpr int kABytes = BM * 128, kBBytes = BN * 128, kSfBytes = 2048;
-constexpr int kStageBytes = kABytes + kBBytes + 2 * kSfBytes;
+constexpr int kTile = 128 * 128, kSf = 2048;
 constexpr int kThreads = 192;
-constexpr int kTmemCols = 256;                // 128 accumulator + 2 x 32 scale-factor columns
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+template <int NB>
+struct Cfg {
+    static constexpr int kStageBytes = kTile * (1 + NB) + kSf * (1 + NB);
+    static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 256;
+    static constexpr int kSfCols = 16 * (1 + NB);                 // per scale-factor buffer
+    static constexpr int kTmemCols = (128 * NB + 2 * kSfCols) <= 256 ? 256 : 512;
+};
 }  // namespace w4a4
 
 struct GemmArgs {
-    int64_t M, N, K;
-    const uint8_t* sfa;   // activation scales, TILED layout for M rows
-    const uint8_t* sfb;   // weight scales, TILED layout for N rows
+    int64_t M, N, K;           // M: rows of A (padded rows when grouped); N: weight rows per expert
+    const uint8_t* sfa;        // A scales, TILED
+    const uint8_t* sfb;        // B scales, TILED (grouped: expert e at sfb + e * sf_stride)
+    int64_t sf_stride;
     const float* gs_a;
-    const float* gs_b;
+    const float* gs_b;         // [1] or [E]
+    const int32_t* tile_info;  // grouped: per 128-row tile {expert, first output row, real rows}
     void* y;
     int64_t ldy;
+    float* yacc;               // COMBINE: fp32 [T, N] accumulation target
+    const int32_t* tok_of;     // COMBINE: token of each permuted row
+    const float* w_of;         // COMBINE: routing weight of each permuted row
     int* status;
 };
 
-template <typename OutT>
-__global__ void __launch_bounds__(w4a4::kThreads, 2)
+NVFP4_DEV float silu(float g) { return g / (1.0f + expf(-g)); }
+
+template <typename OutT, int EPI, bool GROUPED>
+__global__ void __launch_bounds__(w4a4::kThreads, 1)
     gemm_w4a4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                      const GemmArgs a) {
     using namespace w4a4;
+    constexpr int NB = (EPI == NVFP4_EPI_SWIGLU) ? 2 : 1;
+    using C = Cfg<NB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * C::kStageBytes);
     uint64_t* empty = full + kStages;
     uint64_t* accum = empty + kStages;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(accum + 1);
 
+    // tile -> expert, output rows (uniform for the CTA; exits before any setup)
+    int expert = 0, nvalid;
+    int64_t out_row0;
+    const int64_t m0 = (int64_t)blockIdx.x * BM;
+    if constexpr (GROUPED) {
+        const int32_t* ti = a.tile_info + 3 * (int64_t)blockIdx.x;
+        expert = ti[0];
+        if (expert < 0) return;
+        out_row0 = ti[1];
+        nvalid = ti[2];
+    } else {
+        out_row0 = m0;
+        nvalid = (int)((a.M - m0) < BM ? (a.M - m0) : BM);
+    }
+    const int64_t col0 = (int64_t)blockIdx.y * BN;  // output column tile (SWIGLU: of N/2)
+    int64_t brow[NB];                               // first weight row of each B tile, within the expert
+    if constexpr (EPI == NVFP4_EPI_SWIGLU) {
+        brow[0] = col0;
+        brow[NB - 1] = a.N / 2 + col0;
+    } else {
+        brow[0] = col0;
+    }
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t m0 = (int64_t)blockIdx.x * BM, n0 = (int64_t)blockIdx.y * BN;
     const int nk = (int)(a.K / BK);
-    const int64_t cp4 = a.K / 64;   // scale atoms per 128 rows
+    const int64_t cp4 = a.K / 64;  // scale atoms per 128 rows
 
     if (warp == 0) {
-        tmem_alloc(s_tmem, kTmemCols);
+        tmem_alloc(s_tmem, C::kTmemCols);
         tmem_relinquish();
     }
     if (threadIdx.x == 32) {
@@ -92,16 +137,23 @@ __global__ void __launch_bounds__(w4a4::kThreads, 2)
             prefetch_tensormap(&map_a);
             prefetch_tensormap(&map_b);
             const uint8_t* sfa = a.sfa + (m0 / 128) * cp4 * 512;
-            const uint8_t* sfb = a.sfb + (n0 / 128) * cp4 * 512;
+            const uint8_t* sfb_e = a.sfb + (int64_t)expert * a.sf_stride;
             for (int kt = 0; kt < nk; ++kt) {
                 const int slot = kt % kStages;
                 if (kt >= kStages && !mbar_wait(&empty[slot], ((kt / kStages) - 1) & 1, a.status)) break;
-                uint8_t* st = smem + slot * kStageBytes;
-                mbar_expect_tx(&full[slot], kStageBytes);
+                uint8_t* st = smem + slot * C::kStageBytes;
+                mbar_expect_tx(&full[slot], C::kStageBytes);
                 tma_load_2d(st, &map_a, &full[slot], kt * 128, (int)m0);
-                tma_load_2d(st + kABytes, &map_b, &full[slot], kt * 128, (int)n0);
-                bulk_load(st + kABytes + kBBytes, sfa + (int64_t)kt * 4 * 512, kSfBytes, &full[slot]);
-                bulk_load(st + kABytes + kBBytes + kSfBytes, sfb + (int64_t)kt * 4 * 512, kSfBytes, &full[slot]);
+#pragma unroll
+                for (int b = 0; b < NB; ++b)
+                    tma_load_2d(st + kTile * (1 + b), &map_b, &full[slot], kt * 128,
+                                (int)((int64_t)expert * a.N + brow[b]));
+                uint8_t* sf = st + kTile * (1 + NB);
+                bulk_load(sf, sfa + (int64_t)kt * 4 * 512, kSf, &full[slot]);
+#pragma unroll
+                for (int b = 0; b < NB; ++b)
+                    bulk_load(sf + kSf * (1 + b), sfb_e + ((brow[b] / 128) * cp4 + (int64_t)kt * 4) * 512, kSf,
+                              &full[slot]);
             }
         }
     } else if (warp == 1) {
@@ -115,17 +167,17 @@ __global__ void __launch_bounds__(w4a4::kThreads, 2)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t st = smem_u32(smem + slot * kStageBytes);
-                const uint32_t sf_col = 128 + (kt & 1) * 32;   // double-buffered scale-factor columns
-                for (int j = 0; j < 4; ++j) {
-                    tmem_cp_sf_atom(tmem + sf_col + 4 * j, sdesc_sf_atom(st + kABytes + kBBytes + 512 * j));
-                    tmem_cp_sf_atom(tmem + sf_col + 16 + 4 * j,
-                                    sdesc_sf_atom(st + kABytes + kBBytes + kSfBytes + 512 * j));
-                }
-                for (int j = 0; j < 4; ++j) {
-                    mma_nvf4(tmem, sdesc_sw128_kmajor(st + 32 * j), sdesc_sw128_kmajor(st + kABytes + 32 * j), idesc,
-                             tmem + sf_col + 4 * j, tmem + sf_col + 16 + 4 * j, (kt > 0 || j > 0) ? 1u : 0u);
-                }
+                const uint32_t st = smem_u32(smem + slot * C::kStageBytes);
+                const uint32_t sf = st + kTile * (1 + NB);
+                const uint32_t sf_col = 128 * NB + (kt & 1) * C::kSfCols;  // double-buffered scale columns
+                for (int j = 0; j < 4; ++j)
+                    for (int b = 0; b <= NB; ++b)  // b = 0: A's atoms, b >= 1: B tile b-1's atoms
+                        tmem_cp_sf_atom(tmem + sf_col + 16 * b + 4 * j, sdesc_sf_atom(sf + kSf * b + 512 * j));
+                for (int b = 0; b < NB; ++b)
+                    for (int j = 0; j < 4; ++j)
+                        mma_nvf4(tmem + 128 * b, sdesc_sw128_kmajor(st + 32 * j),
+                                 sdesc_sw128_kmajor(st + kTile * (1 + b) + 32 * j), idesc, tmem + sf_col + 4 * j,
+                                 tmem + sf_col + 16 * (1 + b) + 4 * j, (kt > 0 || j > 0) ? 1u : 0u);
                 tc_commit(&empty[slot]);
             }
             if (ok) tc_commit(accum);
@@ -135,38 +187,75 @@ __global__ void __launch_bounds__(w4a4::kThreads, 2)
         const int q = warp & 3;
         const bool ok = mbar_wait(accum, 0, a.status);
         tc_fence_after();
-        const float g = ok ? a.gs_a[0] * a.gs_b[0] : 0.0f;
-        const int64_t row = m0 + 32 * q + lane;
-        OutT* yrow = reinterpret_cast<OutT*>(a.y) + row * a.ldy;
+        const int i = 32 * q + lane;  // row within the tile
+        const bool row_ok = ok && i < nvalid;
+        const float g = ok ? a.gs_a[0] * a.gs_b[GROUPED ? expert : 0] : 0.0f;
+        const int64_t orow = out_row0 + i;
+        int64_t tok = 0;
+        float wgt = 0.0f;
+        if constexpr (EPI == NVFP4_EPI_COMBINE) {
+            if (row_ok) {
+                tok = a.tok_of[orow];
+                wgt = a.w_of[orow];
+            }
+        }
+        const int64_t ncols = (EPI == NVFP4_EPI_SWIGLU) ? a.N / 2 : a.N;
         for (int c0 = 0; c0 < BN; c0 += 32) {
             uint32_t r[32];
             tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + c0, r);
-            tmem_ld_wait();
-            if (!ok || row >= a.M) continue;
-            const int64_t col = n0 + c0;
-            if (col + 32 <= a.N && (a.ldy & 7) == 0) {
-                if constexpr (sizeof(OutT) == 4) {
+            if constexpr (EPI == NVFP4_EPI_SWIGLU) {
+                uint32_t u[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + 128 + c0, u);
+                tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4*>(yrow + col + i) =
-                            make_float4(__uint_as_float(r[i]) * g, __uint_as_float(r[i + 1]) * g,
-                                        __uint_as_float(r[i + 2]) * g, __uint_as_float(r[i + 3]) * g);
+                for (int t = 0; t < 32; ++t)
+                    r[t] = __float_as_uint(silu(__uint_as_float(r[t]) * g) * (__uint_as_float(u[t]) * g));
+            } else {
+                tmem_ld_wait();
+#pragma unroll
+                for (int t = 0; t < 32; ++t) r[t] = __float_as_uint(__uint_as_float(r[t]) * g);
+            }
+            if (!row_ok) continue;
+            const int64_t col = col0 + c0;
+            if constexpr (EPI == NVFP4_EPI_COMBINE) {
+                float* yr = a.yacc + tok * a.ldy + col;
+                if (col + 32 <= ncols && (a.ldy & 3) == 0) {
+#pragma unroll
+                    for (int t = 0; t < 32; t += 4)
+                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(yr + t),
+                                     "f"(wgt * __uint_as_float(r[t])), "f"(wgt * __uint_as_float(r[t + 1])),
+                                     "f"(wgt * __uint_as_float(r[t + 2])), "f"(wgt * __uint_as_float(r[t + 3]))
+                                     : "memory");
                 } else {
-#pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[i + 2 * u]) * g,
-                                                                            __uint_as_float(r[i + 2 * u + 1]) * g);
-                            w[u] = *reinterpret_cast<const uint32_t*>(&b2);
-                        }
-                        *reinterpret_cast<uint4*>(yrow + col + i) = make_uint4(w[0], w[1], w[2], w[3]);
-                    }
+                    for (int t = 0; t < 32; ++t)
+                        if (col + t < ncols) atomicAdd(yr + t, wgt * __uint_as_float(r[t]));
                 }
             } else {
-                for (int i = 0; i < 32; ++i)
-                    if (col + i < a.N) store_out<OutT>(yrow + col + i, __uint_as_float(r[i]) * g);
+                OutT* yrow = reinterpret_cast<OutT*>(a.y) + orow * a.ldy;
+                if (col + 32 <= ncols && (a.ldy & 7) == 0) {
+                    if constexpr (sizeof(OutT) == 4) {
+#pragma unroll
+                        for (int t = 0; t < 32; t += 4)
+                            *reinterpret_cast<float4*>(yrow + col + t) =
+                                make_float4(__uint_as_float(r[t]), __uint_as_float(r[t + 1]),
+                                            __uint_as_float(r[t + 2]), __uint_as_float(r[t + 3]));
+                    } else {
+#pragma unroll
+                        for (int t = 0; t < 32; t += 8) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int u2 = 0; u2 < 4; ++u2) {
+                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[t + 2 * u2]),
+                                                                                __uint_as_float(r[t + 2 * u2 + 1]));
+                                w[u2] = *reinterpret_cast<const uint32_t*>(&b2);
+                            }
+                            *reinterpret_cast<uint4*>(yrow + col + t) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                } else {
+                    for (int t = 0; t < 32; ++t)
+                        if (col + t < ncols) store_out<OutT>(yrow + col + t, __uint_as_float(r[t]));
+                }
             }
         }
     }
@@ -174,18 +263,22 @@ __global__ void __launch_bounds__(w4a4::kThreads, 2)
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc(tmem, C::kTmemCols);
     }
 }
 
-template <typename OutT>
-static int launch_typed(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& a, cudaStream_t st) {
+template <typename OutT, int EPI, bool GROUPED>
+static int launch_typed(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& a, int64_t m_tiles,
+                        cudaStream_t st) {
     using namespace w4a4;
-    auto kern = gemm_w4a4_kernel<OutT>;
+    constexpr int NB = (EPI == NVFP4_EPI_SWIGLU) ? 2 : 1;
+    auto kern = gemm_w4a4_kernel<OutT, EPI, GROUPED>;
     static std::once_flag once;
-    std::call_once(once, [&] { cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes); });
-    dim3 grid((unsigned)((a.M + BM - 1) / BM), (unsigned)((a.N + BN - 1) / BN));
-    kern<<<grid, kThreads, kSmemBytes, st>>>(ma, mb, a);
+    std::call_once(once,
+                   [&] { cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<NB>::kSmemBytes); });
+    const int64_t ncols = (EPI == NVFP4_EPI_SWIGLU) ? a.N / 2 : a.N;
+    dim3 grid((unsigned)m_tiles, (unsigned)((ncols + BN - 1) / BN));
+    kern<<<grid, kThreads, Cfg<NB>::kSmemBytes, st>>>(ma, mb, a);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 
@@ -207,8 +300,48 @@ int launch_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales, const floa
     a.y = y;
     a.ldy = N;
     a.status = status;
-    if (y_dtype == NVFP4_DTYPE_BF16) return launch_typed<__nv_bfloat16>(ma, mb, a, st);
-    return launch_typed<float>(ma, mb, a, st);
+    const int64_t mt = (M + w4a4::BM - 1) / w4a4::BM;
+    if (y_dtype == NVFP4_DTYPE_BF16) return launch_typed<__nv_bfloat16, NVFP4_EPI_NONE, false>(ma, mb, a, mt, st);
+    return launch_typed<float, NVFP4_EPI_NONE, false>(ma, mb, a, mt, st);
+}
+
+int launch_gemm_w4a4_grouped(const uint8_t* a_codes, const uint8_t* a_scales, const float* gs_a, int64_t rows_pad,
+                             int64_t K, const int32_t* tile_info, const uint8_t* w_codes, const uint8_t* w_scales,
+                             int64_t sf_stride, const float* w_gs, int32_t E, int64_t N, int epilogue, void* y,
+                             int y_dtype, float* yacc, const int32_t* tok_of, const float* w_of, int* status,
+                             cudaStream_t st) {
+    CUtensorMap ma, mb;
+    if (!make_tmap_2d_u8(&ma, a_codes, (uint64_t)(K / 2), (uint64_t)rows_pad, 128, w4a4::BM, 1)) return NVFP4_ERR_LAUNCH;
+    if (!make_tmap_2d_u8(&mb, w_codes, (uint64_t)(K / 2), (uint64_t)E * (uint64_t)N, 128, w4a4::BN, 1))
+        return NVFP4_ERR_LAUNCH;
+    GemmArgs a{};
+    a.M = rows_pad;
+    a.N = N;
+    a.K = K;
+    a.sfa = a_scales;
+    a.sfb = w_scales;
+    a.sf_stride = sf_stride;
+    a.gs_a = gs_a;
+    a.gs_b = w_gs;
+    a.tile_info = tile_info;
+    a.y = y;
+    a.yacc = yacc;
+    a.tok_of = tok_of;
+    a.w_of = w_of;
+    a.status = status;
+    const int64_t mt = rows_pad / w4a4::BM;
+    if (epilogue == NVFP4_EPI_SWIGLU) {
+        a.ldy = N / 2;
+        if (y_dtype == NVFP4_DTYPE_BF16) return launch_typed<__nv_bfloat16, NVFP4_EPI_SWIGLU, true>(ma, mb, a, mt, st);
+        return launch_typed<float, NVFP4_EPI_SWIGLU, true>(ma, mb, a, mt, st);
+    }
+    if (epilogue == NVFP4_EPI_COMBINE) {
+        a.ldy = N;
+        return launch_typed<float, NVFP4_EPI_COMBINE, true>(ma, mb, a, mt, st);
+    }
+    a.ldy = N;
+    if (y_dtype == NVFP4_DTYPE_BF16) return launch_typed<__nv_bfloat16, NVFP4_EPI_NONE, true>(ma, mb, a, mt, st);
+    return launch_typed<float, NVFP4_EPI_NONE, true>(ma, mb, a, mt, st);
 }
 
 }  // namespace nvfp4

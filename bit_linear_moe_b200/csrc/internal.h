@@ -9,9 +9,14 @@ namespace nvfp4 {
 
 // quantize.cu
 int launch_amax(const void* x, int x_dtype, int64_t n, unsigned* amax_bits, cudaStream_t st);
+// src_rows (nullable): dst row r quantizes source row src_rows[r]; -1 = zero row.
+// row_bound (nullable, device): rows >= *row_bound are skipped entirely.
 int launch_quantize(const void* x, int x_dtype, const int32_t* src_rows, int64_t dst_rows, int64_t cols,
                     int sf_layout, const float* gs_in, const unsigned* amax_bits, uint8_t* codes,
-                    uint8_t* scales, float* gs_out, cudaStream_t st);
+                    uint8_t* scales, float* gs_out, cudaStream_t st, const int32_t* row_bound = nullptr);
+// amax over bf16 rows x[src_rows[r]], r < nrows (negative entries skipped).
+int launch_amax_rows(const void* x, const int32_t* src_rows, int64_t nrows, int64_t cols, unsigned* amax_bits,
+                     cudaStream_t st);
 
 // gemv.cu: W4A16 on CUDA cores.
 struct GemvArgs {
@@ -60,6 +65,22 @@ int launch_perm_scatter(const int32_t* topk_idx, int64_t T, int32_t E, int32_t k
                         int32_t* perm_tok, int32_t* perm_slot, int32_t* row_of, cudaStream_t st);
 int launch_combine(const float* d, const float* topk_w, const int32_t* row_of, int64_t T, int32_t k, int64_t N,
                    void* y, int y_dtype, cudaStream_t st);
+
+// Padded expert layout (rows_pad = multiple of 128 >= R + 127 E): pad_off[E+1],
+// tile_info[3 * rows_pad/128], src_rows[rows_pad].
+int launch_moe_pad(const int32_t* offsets, int32_t E, int64_t rows_pad, const int32_t* gather, int32_t* pad_off,
+                   int32_t* tile_info, int32_t* src_rows, cudaStream_t st);
+int launch_f32_to_bf16(const float* src, int64_t n, void* dst, cudaStream_t st);  // n % 4 == 0
+// tok_of[row_of[i]] = i / k, w_of[row_of[i]] = topk_w[i] for i < n (= T * k).
+int launch_row_token(const int32_t* row_of, const float* topk_w, int64_t n, int32_t k, int32_t* tok_of, float* w_of,
+                     cudaStream_t st);
+
+// gemm_w4a4.cu, grouped: A = padded permuted activations, B = stacked experts.
+int launch_gemm_w4a4_grouped(const uint8_t* a_codes, const uint8_t* a_scales, const float* gs_a, int64_t rows_pad,
+                             int64_t K, const int32_t* tile_info, const uint8_t* w_codes, const uint8_t* w_scales,
+                             int64_t sf_stride, const float* w_gs, int32_t E, int64_t N, int epilogue, void* y,
+                             int y_dtype, float* yacc, const int32_t* tok_of, const float* w_of, int* status,
+                             cudaStream_t st);
 
 constexpr int kPermBlockTokens = 128;
 

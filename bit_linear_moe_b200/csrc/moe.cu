@@ -239,7 +239,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
         const float wj = w[t * k + j];
-        const float4 v = *reinterpret_cast<const float4*>(d + (int64_t)row_of[t * k + j] * N + c);
+        const int32_t r = row_of[t * k + j];
+        if (r < 0 || (int64_t)r >= T * k) continue;  // row_of must index the T * k rows of d
+        const float4 v = *reinterpret_cast<const float4*>(d + (int64_t)r * N + c);
         acc.x = fmaf(wj, v.x, acc.x);
         acc.y = fmaf(wj, v.y, acc.y);
         acc.z = fmaf(wj, v.z, acc.z);
@@ -259,6 +261,118 @@ int launch_combine(const float* d, const float* topk_w, const int32_t* row_of, i
         combine_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(d, topk_w, row_of, T, k, N, (__nv_bfloat16*)y);
     else
         combine_kernel<float><<<grid, 256, 0, st>>>(d, topk_w, row_of, T, k, N, (float*)y);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+}
+
+}  // namespace nvfp4
+
+namespace nvfp4 {
+
+// ---- padded expert layout for the grouped tensor-core GEMM ------------------
+// Each expert's rows are padded to whole 128-row tiles.  pad_off[e] is the
+// first padded row of expert e; tile_info[t] = {expert, first output row,
+// real rows} for the used tiles and {-1, 0, 0} for the rest.
+__global__ void __launch_bounds__(1024) moe_pad_kernel(const int32_t* __restrict__ offsets, int32_t E,
+                                                       int64_t n_mtiles, int32_t* __restrict__ pad_off,
+                                                       int32_t* __restrict__ tile_info) {
+    __shared__ int32_t tiles[kMaxE];
+    const int e = threadIdx.x;
+    const int32_t cnt = e < E ? offsets[e + 1] - offsets[e] : 0;
+    const int32_t mine = (cnt + 127) / 128;
+    tiles[e] = mine;
+    __syncthreads();
+    for (int o = 1; o < kMaxE; o <<= 1) {
+        const int32_t add = e >= o ? tiles[e - o] : 0;
+        __syncthreads();
+        tiles[e] += add;
+        __syncthreads();
+    }
+    const int32_t first = tiles[e] - mine;
+    const int32_t total = tiles[kMaxE - 1];
+    if (e < E) {
+        pad_off[e] = first * 128;
+        for (int32_t t = 0; t < mine; ++t) {
+            int32_t* ti = tile_info + 3 * (int64_t)(first + t);
+            ti[0] = e;
+            ti[1] = offsets[e] + 128 * t;
+            ti[2] = min(128, cnt - 128 * t);
+        }
+    }
+    if (e == 0) pad_off[E] = total * 128;
+    for (int64_t t = total + e; t < n_mtiles; t += blockDim.x) {
+        int32_t* ti = tile_info + 3 * t;
+        ti[0] = -1;
+        ti[1] = 0;
+        ti[2] = 0;
+    }
+}
+
+// src_rows[pr] = activation row read by padded row pr (-1 for padding).
+__global__ void __launch_bounds__(256) moe_src_rows_kernel(const int32_t* __restrict__ pad_off,
+                                                           const int32_t* __restrict__ offsets, int32_t E,
+                                                           const int32_t* __restrict__ gather, int64_t rows_pad,
+                                                           int32_t* __restrict__ src_rows) {
+    const int64_t pr = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (pr >= rows_pad) return;
+    int32_t src = -1;
+    if (pr < pad_off[E]) {
+        int lo = 0, hi = E;  // last e with pad_off[e] <= pr
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) / 2;
+            if (pad_off[mid] <= pr) lo = mid; else hi = mid;
+        }
+        const int64_t local = pr - pad_off[lo];
+        const int32_t cnt = offsets[lo + 1] - offsets[lo];
+        if (local < cnt) {
+            const int64_t r = offsets[lo] + local;
+            src = gather ? gather[r] : (int32_t)r;
+        }
+    }
+    src_rows[pr] = src;
+}
+
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restrict__ src, int64_t n4,
+                                                          __nv_bfloat16* __restrict__ dst) {
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= n4) return;
+    const float4 v = reinterpret_cast<const float4*>(src)[i];
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&a);
+    o.y = *reinterpret_cast<const uint32_t*>(&b);
+    reinterpret_cast<uint2*>(dst)[i] = o;
+}
+
+// Inverse of row_of for the combine epilogue: tok_of[row] = token, w_of[row] = its routing weight.
+__global__ void __launch_bounds__(256) row_token_kernel(const int32_t* __restrict__ row_of,
+                                                        const float* __restrict__ topk_w, int64_t n, int32_t k,
+                                                        int32_t* __restrict__ tok_of, float* __restrict__ w_of) {
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const int32_t r = row_of[i];
+    if (r < 0 || (int64_t)r >= n) return;  // row_of must be a permutation of [0, n)
+    tok_of[r] = (int32_t)(i / k);
+    w_of[r] = topk_w[i];
+}
+
+int launch_row_token(const int32_t* row_of, const float* topk_w, int64_t n, int32_t k, int32_t* tok_of, float* w_of,
+                     cudaStream_t st) {
+    row_token_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(row_of, topk_w, n, k, tok_of, w_of);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+}
+
+int launch_moe_pad(const int32_t* offsets, int32_t E, int64_t rows_pad, const int32_t* gather, int32_t* pad_off,
+                   int32_t* tile_info, int32_t* src_rows, cudaStream_t st) {
+    moe_pad_kernel<<<1, kMaxE, 0, st>>>(offsets, E, rows_pad / 128, pad_off, tile_info);
+    if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
+    moe_src_rows_kernel<<<(unsigned)((rows_pad + 255) / 256), 256, 0, st>>>(pad_off, offsets, E, gather, rows_pad,
+                                                                            src_rows);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+}
+
+int launch_f32_to_bf16(const float* src, int64_t n, void* dst, cudaStream_t st) {
+    const int64_t n4 = n / 4;
+    f32_to_bf16_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(src, n4, (__nv_bfloat16*)dst);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 

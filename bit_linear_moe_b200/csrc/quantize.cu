@@ -70,6 +70,32 @@ __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int6
     }
 }
 
+// max|x| over the rows src_rows[r] (r < nrows, entries < 0 skipped), 16 columns per item.
+template <typename T>
+__global__ void __launch_bounds__(256) amax_rows_kernel(const T* __restrict__ x, const int32_t* __restrict__ src_rows,
+                                                        int64_t nrows, int64_t cols, unsigned* __restrict__ amax_bits) {
+    float m = 0.0f;
+    const int64_t nb = cols / 16, n = nrows * nb;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / nb, b = i % nb;
+        const int32_t src = src_rows[r];
+        if (src < 0) continue;
+        float v[16];
+        Vec16<T>::load(x + (int64_t)src * cols + b * 16, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(v[j]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    __shared__ float red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+        atomicMax(amax_bits, __float_as_uint(m));
+    }
+}
+
 NVFP4_DEV float global_scale_from(const float* gs_in, const unsigned* amax_bits) {
     if (gs_in) return *gs_in;
     const float amax = __uint_as_float(*amax_bits);
@@ -85,12 +111,13 @@ __global__ void __launch_bounds__(256) quantize_kernel(
     const T* __restrict__ x, const int32_t* __restrict__ src_rows, int64_t dst_rows, int64_t cols,
     int64_t grid_rows, int64_t grid_cols, const float* __restrict__ gs_in,
     const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-    float* __restrict__ gs_out) {
+    float* __restrict__ gs_out, const int32_t* __restrict__ row_bound) {
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     const float gs = global_scale_from(gs_in, amax_bits);
     if (i == 0 && gs_out) *gs_out = gs;
     if (i >= grid_rows * grid_cols) return;
     const int64_t r = i / grid_cols, b = i % grid_cols;
+    if (row_bound && r >= (int64_t)*row_bound) return;  // rows nobody reads (padded expert layout)
     const int64_t nsf = cols >> 4;
     const int64_t soff = sf_offset<LAYOUT>(r, b, nsf);
     int64_t src = r;
@@ -141,16 +168,25 @@ int launch_amax(const void* x, int x_dtype, int64_t n, unsigned* amax_bits, cuda
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 
+int launch_amax_rows(const void* x, const int32_t* src_rows, int64_t nrows, int64_t cols, unsigned* amax_bits,
+                     cudaStream_t st) {
+    if (cudaMemsetAsync(amax_bits, 0, sizeof(unsigned), st) != cudaSuccess) return NVFP4_ERR_LAUNCH;
+    int grid = grid_for(nrows * (cols / 16), 256);
+    if (grid > 148 * 8) grid = 148 * 8;
+    amax_rows_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, src_rows, nrows, cols, amax_bits);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+}
+
 int launch_quantize(const void* x, int x_dtype, const int32_t* src_rows, int64_t dst_rows, int64_t cols,
                     int sf_layout, const float* gs_in, const unsigned* amax_bits, uint8_t* codes,
-                    uint8_t* scales, float* gs_out, cudaStream_t st) {
+                    uint8_t* scales, float* gs_out, cudaStream_t st, const int32_t* row_bound) {
     const int64_t nsf = cols / 16;
     const int64_t grid_rows = sf_layout == NVFP4_SF_TILED ? (dst_rows + 127) / 128 * 128 : dst_rows;
     const int64_t grid_cols = sf_layout == NVFP4_SF_TILED ? (nsf + 3) / 4 * 4 : nsf;
     const int grid = grid_for(grid_rows * grid_cols, 256);
 #define NVFP4_Q(T, L)                                                                                 \
     quantize_kernel<T, L><<<grid, 256, 0, st>>>((const T*)x, src_rows, dst_rows, cols, grid_rows,     \
-                                                grid_cols, gs_in, amax_bits, codes, scales, gs_out)
+                                                grid_cols, gs_in, amax_bits, codes, scales, gs_out, row_bound)
     if (x_dtype == NVFP4_DTYPE_BF16) {
         if (sf_layout == NVFP4_SF_TILED) NVFP4_Q(__nv_bfloat16, NVFP4_SF_TILED);
         else NVFP4_Q(__nv_bfloat16, NVFP4_SF_ROWMAJOR);

@@ -166,3 +166,87 @@ def test_untouched_experts_are_not_read():
                                perm_tok=dev["perm_tok"], epilogue=nv.EPI_SWIGLU, mode=nv.MODE_W4A16)
     torch.cuda.synchronize()
     assert torch.isfinite(a2).all() and torch.equal(a1, a2)
+
+
+# ---- grouped W4A4 (tensor-core) expert layer ---------------------------------
+
+def _w4a4_layer(E, T, zipf_like, seed=20):
+    """E experts with the per-expert shapes of the 512-expert layer; weights
+    quantized on the GPU (bit-exactness of that quantizer is tested in
+    test_gpu_quantize) and by the oracle for the experts it checks."""
+    rng = np.random.default_rng(seed)
+    wr = synth.to_bf16(0.02 * rng.standard_normal((E, H)))
+    h = synth.activations(np.random.default_rng([seed, T]), T, H)
+    bias = (-1.1 * np.log(np.random.default_rng([seed, 1]).permutation(E) + 1)).astype(np.float32) if zipf_like \
+        else None
+    gu_f = [synth.weight(np.random.default_rng([seed, 2, e]), 2 * I, H) for e in range(E)]
+    dn_f = [synth.weight(np.random.default_rng([seed, 3, e]), H, I) for e in range(E)]
+
+    def stack(ws):
+        N, K = ws[0].shape
+        sb = nv.nvfp4_scales_bytes(N, K, nv.SF_TILED)
+        codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device="cuda")
+        scales = torch.empty(E * sb, dtype=torch.uint8, device="cuda")
+        gs = torch.empty(E, dtype=torch.float32, device="cuda")
+        for e, w in enumerate(ws):
+            nv.nvfp4_quantize(torch.from_numpy(w).cuda(), sf_layout=nv.SF_TILED, codes=codes[e],
+                              scales=scales[e * sb:(e + 1) * sb], gs_out=gs[e:e + 1])
+        return codes, scales, gs
+
+    return h, wr, bias, gu_f, dn_f, stack(gu_f), stack(dn_f)
+
+
+@pytest.mark.parametrize("zipf", [False, True])
+def test_expert_layer_w4a4_4096_tokens(zipf):
+    E_, T = 64, 4096
+    h, wr, bias, gu_f, dn_f, (gc, gsc, ggs), (dc, dsc, dgs) = _w4a4_layer(E_, T, zipf)
+    hd = torch.from_numpy(h).to(torch.bfloat16).cuda()
+    out = nv.moe_route_topk(hd, torch.from_numpy(wr).to(torch.bfloat16).cuda(), K_TOP,
+                            logit_bias=None if bias is None else torch.from_numpy(bias).cuda())
+    R = T * K_TOP
+    a = nv.moe_grouped_linear(hd, out["expert_offsets"], gc, gsc, ggs, R, perm_tok=out["perm_tok"], gather=True,
+                              w_sf_layout=nv.SF_TILED, epilogue=nv.EPI_SWIGLU, y_dtype=torch.bfloat16,
+                              mode=nv.MODE_W4A4)
+    y = nv.moe_grouped_linear(a, out["expert_offsets"], dc, dsc, dgs, R, gather=False, w_sf_layout=nv.SF_TILED,
+                              epilogue=nv.EPI_COMBINE, topk_w=out["topk_w"], row_of=out["row_of"], k=K_TOP,
+                              y_dtype=torch.float32, mode=nv.MODE_W4A4)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_read_device_status() == nv.OK
+    g = {k2: v.cpu().numpy() for k2, v in out.items()}
+    a_np = a.float().cpu().numpy()
+    y_np = y.cpu().numpy()
+    off, pt, row_of, tw = g["expert_offsets"], g["perm_tok"], g["row_of"], g["topk_w"].astype(np.float64)
+    expert_of_row = np.searchsorted(off, np.arange(R), side="right") - 1
+    toks = np.sort(np.random.default_rng(5).choice(T, 24, replace=False))
+    gs_h = oracle.global_scale(h)
+    gs_a = oracle.global_scale(a_np)
+    q_gu, q_dn = {}, {}
+    for t in toks:
+        for j in range(K_TOP):
+            r = int(row_of[t, j])
+            e = int(expert_of_row[r])
+            if e not in q_gu:
+                q_gu[e] = oracle.quantize(gu_f[e])
+                q_dn[e] = oracle.quantize(dn_f[e])
+            # stage 1: gate/up (W4A4 on the gathered, quantized hidden state) + SwiGLU
+            xq = oracle.quantize(h[pt[r]:pt[r] + 1], gs=gs_h)
+            gu, gu_ad = oracle.linear_w4a4(xq, q_gu[e])
+            ref_a = omoe.swiglu(gu)[0]
+            gg, uu = gu[0, :I], gu[0, I:]
+            sig = 1.0 / (1.0 + np.exp(-gg))
+            dg, du = 1e-4 * gu_ad[0, :I] + 1e-6, 1e-4 * gu_ad[0, I:] + 1e-6
+            bound = (np.abs(uu) * np.abs(sig * (1 + gg * (1 - sig))) * dg + np.abs(gg * sig) * du + dg * du
+                     + 1e-5 * np.abs(ref_a) + 1e-6 + bf16_ulp(ref_a))
+            err = np.abs(a_np[r] - ref_a)
+            assert (err <= bound).all(), f"swiglu row {r}: max ratio {np.max(err / bound)}"
+        # stage 2: down projection of the GPU's own a, then the weighted combine
+        ref_y = np.zeros(H)
+        ref_b = np.zeros(H)
+        for j in range(K_TOP):
+            r = int(row_of[t, j])
+            e = int(expert_of_row[r])
+            aq = oracle.quantize(a_np[r:r + 1], gs=gs_a)
+            d, d_ad = oracle.linear_w4a4(aq, q_dn[e])
+            ref_y += tw[t, j] * d[0]
+            ref_b += abs(tw[t, j]) * d_ad[0]
+        assert_within_bound(y_np[t], ref_y, ref_b, False, f"down+combine token {t}")
