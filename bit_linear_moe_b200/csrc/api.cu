@@ -3,6 +3,7 @@
 // include/nvfp4.h.  Every entry point validates on the host and returns an
 // error before launching anything.
 #include <cuda_runtime.h>
+#include <stdlib.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -25,6 +26,14 @@ static int* device_status_ptr() {
     return cache[dev];
 }
 static size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char* e = getenv("NVFP4_PDL");
+        return !(e && e[0] == '0');
+    }();
+    return on;
+}
 
 // The current device must be sm_100 (B200 / GB200 class).  Cached per device.
 static int check_arch() {
@@ -230,6 +239,8 @@ int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t
     void* xh = ws;
     float* inv = (float*)((char*)ws + align256((size_t)(M * K) * 2));
     NVFP4_TRY(launch_x_prep(x, nullptr, M, K, xh, inv, st));
+    if (w4a16_tc_supported(M, K, N, w_sf_layout))
+        return launch_w4a16_tc(xh, inv, M, K, w_codes, w_scales, w_gs, N, y, y_dtype, device_status_ptr(), st);
     GemvArgs a{};
     a.xh = xh;
     a.inv_scale = inv;

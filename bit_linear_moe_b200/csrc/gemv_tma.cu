@@ -1,4 +1,5 @@
-// K2 (pipelined form): W4A16 decode for M <= 4 with K % 256 == 0.
+// K2 (pipelined form): W4A16 decode for M <= 2 with K % 256 == 0 (wider
+// batches go to the tensor-memory kernel in gemm_w4a16_tc.cu).
 //
 // Ignis README, "The decode round": decode linears are weight streaming at
 // the card's bandwidth; this kernel is built so that the HBM stream never
@@ -27,7 +28,9 @@
 // mixed-precision fma.rn.f32.f16.  The K range of a tile is split over a
 // cluster of QS CTAs (QS chosen so that the grid is one wave over the SMs);
 // their partial sums meet through distributed shared memory and rank 0 writes
-// the output.
+// the output.  Launched as a programmatic dependent: the first ring of weight
+// stages is requested before the previous kernel in the stream completes, the
+// activations after it.
 #include <cuda.h>
 
 #include <map>
@@ -136,16 +139,24 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int t = 0; t < MT; ++t) inv_p[t] = 1.0f;
 
+    griddep_launch_dependents();
     if (warp == 8) {
         // ---------------- producer ----------------
         if (lane == 0) {
             prefetch_tensormap(&codes_map);
             if (LAYOUT == NVFP4_SF_ROWMAJOR) prefetch_tensormap(&sc_map);
-            mbar_expect_tx(xbar, (uint32_t)(nt * ns * kStageK * 2));
-            for (int t = 0; t < nt; ++t)
-                bulk_load(s_x + t * kr_max, a.x + (m0 + t) * a.K + k_begin, (uint32_t)(ns * kStageK * 2), xbar);
+            // the first ring's worth of weights goes out before the previous
+            // kernel has finished; the activations only after it
+            const int pre = ns < kStages ? ns : kStages;
             for (int s = 0; s < ns; ++s) {
                 const int slot = s % kStages;
+                if (s == pre) {
+                    griddep_wait();
+                    mbar_expect_tx(xbar, (uint32_t)(nt * ns * kStageK * 2));
+                    for (int t = 0; t < nt; ++t)
+                        bulk_load(s_x + t * kr_max, a.x + (m0 + t) * a.K + k_begin, (uint32_t)(ns * kStageK * 2),
+                                  xbar);
+                }
                 if (s >= kStages) {
                     if (!mbar_wait(&empty[slot], ((s / kStages) - 1) & 1, a.status)) break;
                     fence_proxy_async();  // consumers' generic reads before the async-proxy refill
@@ -159,8 +170,15 @@ __global__ void __launch_bounds__(kThreads, 2)
                 else
                     tma_load_2d(s_scales + slot * kScaleBytes, &sc_map, &full[slot], st * 16, (int)row0);
             }
+            if (ns <= kStages) {
+                griddep_wait();
+                mbar_expect_tx(xbar, (uint32_t)(nt * ns * kStageK * 2));
+                for (int t = 0; t < nt; ++t)
+                    bulk_load(s_x + t * kr_max, a.x + (m0 + t) * a.K + k_begin, (uint32_t)(ns * kStageK * 2), xbar);
+            }
         }
     } else {
+        griddep_wait();
         // ---------------- consumers ----------------
         const int ch = lane & 7, rsub = lane >> 3;
         bool ok = mbar_wait(xbar, 0, a.status);
@@ -319,13 +337,14 @@ static int launch_one(const DecodeArgs& a, const CUtensorMap& cm, const CUtensor
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = decode_smem_bytes(MT, kr_max);
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)a.QS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    set_pdl_attr(attr[1]);
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, kern, cm, sm, a) == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 
@@ -392,7 +411,7 @@ static int run_mt(const DecodeArgs& a, const uint8_t* codes, const uint8_t* scal
 }
 
 bool decode_tma_supported(int64_t M, int64_t K, int64_t N) {
-    return M <= 4 && K % kStageK == 0 && K / 2 <= ((int64_t)1 << 31) && N <= ((int64_t)1 << 31);
+    return M <= 2 && K % kStageK == 0 && K / 2 <= ((int64_t)1 << 31) && N <= ((int64_t)1 << 31);
 }
 
 int launch_decode_tma(const void* x, int64_t M, int64_t K, const uint8_t* codes, const uint8_t* scales,

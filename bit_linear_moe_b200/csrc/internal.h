@@ -7,6 +7,15 @@
 
 namespace nvfp4 {
 
+// Launch attribute for programmatic dependent launch (kernels that call
+// griddep_wait() before touching activations or outputs).  Off when the
+// environment sets NVFP4_PDL=0.
+bool pdl_enabled();
+inline void set_pdl_attr(cudaLaunchAttribute& a) {
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = 1;
+}
+
 // quantize.cu
 int launch_amax(const void* x, int x_dtype, int64_t n, unsigned* amax_bits, cudaStream_t st);
 // src_rows (nullable): dst row r quantizes source row src_rows[r]; -1 = zero row.
@@ -42,6 +51,12 @@ struct GemvArgs {
 int launch_x_prep(const void* x, const int32_t* gather, int64_t rows, int64_t K, void* xh, float* inv_scale,
                   cudaStream_t st);
 int launch_gemv_w4a16(const GemvArgs& a, cudaStream_t st);
+
+// gemm_w4a16_tc.cu: W4A16 with dequantized weights in tensor memory (M <= 32, TILED, K % 256 == 0).
+bool w4a16_tc_supported(int64_t M, int64_t K, int64_t N, int sf_layout);
+int launch_w4a16_tc(const void* xh, const float* inv_scale, int64_t M, int64_t K, const uint8_t* codes,
+                    const uint8_t* scales, const float* gs, int64_t N, void* y, int y_dtype, int* status,
+                    cudaStream_t st);
 
 // gemv_tma.cu: pipelined W4A16 decode (TMA ring, cluster split-K) for M <= 4, K % 256 == 0.
 bool decode_tma_supported(int64_t M, int64_t K, int64_t N);

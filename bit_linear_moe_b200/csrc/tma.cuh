@@ -17,6 +17,17 @@ constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
 
 NVFP4_DEV uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the kernel before it in the stream is still
+// running.  griddep_wait() returns once that kernel has completed and its
+// writes are visible; nothing an earlier kernel may still be writing (the
+// activations) is read, and no output is written, before it.  Weights are
+// read-only for the duration of a forward pass and may be fetched before it.
+// griddep_launch_dependents() lets the next such kernel start as soon as every
+// CTA of this grid has issued it.
+NVFP4_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+NVFP4_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 NVFP4_DEV void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }

@@ -53,7 +53,7 @@ def test_dense27b_decode(name, K, N, seed, M):
     q = _dense_q(seed, K, N)
     x = synth.decode_x(seed, M, K)
     ref, ad = oracle.linear_w4a16(x, *q)
-    layout = nv.SF_TILED if M in (1, 8) else nv.SF_ROWMAJOR
+    layout = nv.SF_ROWMAJOR if M == 2 else nv.SF_TILED
     y = _run(x, q, layout, torch.float32)
     assert_within_bound(y, ref, ad, False, f"{name} M={M}")
     if M == 1:
@@ -87,3 +87,16 @@ def test_degenerate_weights():
     y = _run(x, (codes, scales, np.float32(0.5)), nv.SF_ROWMAJOR, torch.float32).cpu().numpy()
     assert y[0, 5] == np.float32(x[0, 19] * 6.0 * 0.5) and y[1, 5] == np.float32(x[1, 19] * 3.0)
     assert np.count_nonzero(y) == 2
+
+
+@pytest.mark.parametrize("M,K,N", [(5, 256, 128), (8, 512, 200), (13, 1024, 1000), (16, 256, 64), (17, 768, 130),
+                                   (32, 5120, 256), (24, 2048, 384)])
+def test_tensor_core_widths(M, K, N):
+    """Widths 5..32 with tensor-core scales run the tensor-memory kernel."""
+    rng = np.random.default_rng(M * 7 + K + N)
+    q = oracle.quantize(synth.weight(rng, N, K))
+    x = synth.activations(rng, M, K)
+    ref, ad = oracle.linear_w4a16(x, *q)
+    for y_dtype in (torch.float32, torch.bfloat16):
+        y = _run(x, q, nv.SF_TILED, y_dtype)
+        assert_within_bound(y, ref, ad, y_dtype == torch.bfloat16, f"tc {M}x{K}x{N}")
