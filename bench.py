@@ -58,8 +58,9 @@ def load_peaks():
 
 
 def kernel_traffic(kernel_src: str, name: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current source of the kernel (matched by hash); else None."""
+    """DRAM bytes of one decode step (the kernel's 4 launches) from a committed
+    ncu summary, if it was taken on the current source of the kernel (matched
+    by hash); else None."""
     src = os.path.join(ROOT, "bit_linear_moe_b200", "csrc", kernel_src)
     p = os.path.join(ROOT, "profiles", f"{name}.traffic.txt")
     if not (os.path.exists(src) and os.path.exists(p)):
@@ -73,7 +74,7 @@ def kernel_traffic(kernel_src: str, name: str):
     if vals.get("source_sha256_16") != h:
         return None
     try:
-        return float(vals["dram_bytes_per_launch"])
+        return float(vals["dram_bytes_per_step"])
     except (KeyError, ValueError):
         return None
 
@@ -285,6 +286,7 @@ def run_native(args, rank, world, dist):
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
+                     "per": "decode step (4 launches, one per shape); achieved = algorithmic bytes / summed launch time",
                      "kernel": "gemv_tma_kernel (the only launch of each linear): per-shape graph replays timed with CUDA events"},
         "e2e": {"value": round(e2e, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 4 * args.steps,
