@@ -48,6 +48,21 @@ def decode_bytes(M, K, N):
     return N * K // 2 + N * K // 16 + M * K * 2 + 4
 
 
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The slowest rank's time (every rank gets it); ``ms`` unchanged on one rank."""
+    if not dist:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_step: int, ms_per_step: float) -> float:
+    """Aggregate GB/s of `world` replicas that each stream `bytes_per_step` per step."""
+    return world * bytes_per_step / (ms_per_step * 1e-3) / 1e9
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -208,13 +223,9 @@ def run_native(args, rank, world, dist):
             step_graphs[i % 2].replay()
         t1.record(stream)
         torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
-    if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), dist, dev)
     ms_per_step = ms / args.steps
-    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    value = whole_job_gbs(world, step_bytes, ms_per_step)
 
     # per-shape device time: each linear alone, replayed from its graph
     reps = max(200, min(2000, args.steps))
@@ -263,17 +274,15 @@ def run_native(args, rank, world, dist):
         e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
-    e2e = world * step_bytes / (e_ms / args.steps * 1e-3) / 1e9
+    e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev)
+    e2e = whole_job_gbs(world, step_bytes, e_ms / args.steps)
 
     extra = {"decode_m1_per_shape": per_shape}
     if not args.quick:
         extra["decode_sweep"] = decode_sweep(nv, torch, dev, layers)
         extra["prefill"] = prefill_section(nv, torch, dev, layers)
+        extra["quantize"] = quantize_section(nv, torch, dev)
+        extra["moe_layer"] = moe_section(nv, torch, dev)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -404,6 +413,108 @@ def prefill_section(nv, torch, dev, layers, M=2048, reps=30):
     out["with_quant_TFLOPs"] = round(tot_flop / (tot_e2e * 1e-3) / 1e12, 1)
     out["peak_nominal_dense_nvfp4_TFLOPs"] = 9000.0
     out["frac_of_nominal"] = round(out["gemm_TFLOPs"] / 9000.0, 4)
+    return out
+
+
+MOE_EXPERT_BYTES = 1024 * 2048 // 2 + 1024 * 2048 // 16 + 2048 * 512 // 2 + 2048 * 512 // 16  # 1,769,472
+
+
+def moe_section(nv, torch, dev, reps=30):
+    """One mixture-of-experts layer (512 experts, hidden 2048, expert width 512,
+    top-10): route, gather + gate/up + SwiGLU, down + weighted combine.
+    GB/s = (touched experts x 1,769,472 B + T x 2048 x (2 + 4) B for h in and
+    y out) / time; W4A16 at T = 1, 32 and W4A4 at T = 4096, uniform routing
+    and a Zipf(1.1) popularity bias.  Expert weights 0.02 N(0, 1) drawn on the
+    device from a seeded generator and quantized per expert matrix."""
+    from bit_linear_moe_b200 import synth
+    E, H, I, k = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_K
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(10)
+
+    def stack(n, kk):
+        cs, ss, gs = [], [], []
+        for _ in range(E):
+            w = 0.02 * torch.randn((n, kk), generator=gen, device=dev)
+            c, sc, g = nv.nvfp4_quantize(w, sf_layout=nv.SF_TILED)
+            cs.append(c)
+            ss.append(sc)
+            gs.append(g)
+        return torch.stack(cs), torch.stack(ss).reshape(-1), torch.cat(gs)
+
+    gu = stack(2 * I, H)
+    dn = stack(H, I)
+    wr = (0.02 * torch.randn((E, H), generator=gen, device=dev)).to(torch.bfloat16)
+    zipf = torch.from_numpy(synth.moe_zipf_bias()).to(dev)
+    out = {"experts": E, "hidden": H, "expert_width": I, "top_k": k, "bytes_per_touched_expert": MOE_EXPERT_BYTES,
+           "runs": {}}
+    for T, mode, nbatch in ((1, nv.MODE_W4A16, 16), (32, nv.MODE_W4A16, 4), (4096, nv.MODE_W4A4, 2)):
+        R = T * k
+        ws1 = torch.empty(max(16, int(nv.lib().moe_grouped_linear_workspace(R, H, 2 * I, E, k, nv.EPI_SWIGLU, mode))),
+                          dtype=torch.uint8, device=dev)
+        ws2 = torch.empty(max(16, int(nv.lib().moe_grouped_linear_workspace(R, I, H, E, k, nv.EPI_COMBINE, mode))),
+                          dtype=torch.uint8, device=dev)
+        for bias_name, bias in (("uniform", None), ("zipf", zipf)):
+            hs = [torch.randn((T, H), generator=gen, device=dev).to(torch.bfloat16) for _ in range(nbatch)]
+            a = torch.empty((R, I), dtype=torch.bfloat16, device=dev)
+            y = torch.empty((T, H), dtype=torch.float32, device=dev)
+            touched = []
+
+            def layer(i):
+                r = nv.moe_route_topk(hs[i], wr, k, logit_bias=bias)
+                nv.moe_grouped_linear(hs[i], r["expert_offsets"], gu[0], gu[1], gu[2], R, perm_tok=r["perm_tok"],
+                                      gather=True, w_sf_layout=nv.SF_TILED, epilogue=nv.EPI_SWIGLU, y=a,
+                                      mode=mode, ws=ws1)
+                nv.moe_grouped_linear(a, r["expert_offsets"], dn[0], dn[1], dn[2], R, gather=False,
+                                      w_sf_layout=nv.SF_TILED, epilogue=nv.EPI_COMBINE, topk_w=r["topk_w"],
+                                      row_of=r["row_of"], k=k, y=y, mode=mode, ws=ws2)
+                return r
+
+            for i in range(nbatch):
+                r = layer(i)
+                touched.append(int((torch.diff(r["expert_offsets"]) > 0).sum().item()))
+            torch.cuda.synchronize()
+            stream = torch.cuda.current_stream()
+            side = torch.cuda.Stream(device=dev)
+            side.wait_stream(stream)
+            graphs = []
+            with torch.cuda.stream(side):
+                for i in range(nbatch):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=side):
+                        layer(i)
+                    graphs.append(g)
+            stream.wait_stream(side)
+            t = _time_graphs(torch, graphs, max(reps, 2 * nbatch))
+            nbytes = sum(touched) / nbatch * MOE_EXPERT_BYTES + T * H * 6
+            flop = 2.0 * R * (H * 2 * I + I * H)
+            key = f"T{T}_{bias_name}"
+            out["runs"][key] = {"mode": "W4A16" if mode == nv.MODE_W4A16 else "W4A4", "us": round(t * 1e3, 2),
+                                "touched_experts_mean": round(sum(touched) / nbatch, 1),
+                                "GB/s": round(nbytes / (t * 1e-3) / 1e9, 1),
+                                "TFLOPs": round(flop / (t * 1e-3) / 1e12, 2)}
+    del gu, dn
+    return out
+
+
+def quantize_section(nv, torch, dev, reps=30):
+    """Activation quantize (two passes: amax, then scales and codes) of bf16
+    [M, 5120]: GB/s = (2 M K + 2 M K + 0.5625 M K) / time."""
+    out = {}
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    K = 5120
+    for M in (2048, 8192):
+        xs = [torch.randn((M, K), generator=gen, device=dev).to(torch.bfloat16) for _ in range(2)]
+        codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty(int(nv.nvfp4_scales_bytes(M, K, nv.SF_TILED)), dtype=torch.uint8, device=dev)
+        gs = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.empty(max(16, int(nv.lib().nvfp4_quantize_workspace(M, K))), dtype=torch.uint8, device=dev)
+
+        def q(i):
+            nv.nvfp4_quantize(xs[i], sf_layout=nv.SF_TILED, codes=codes, scales=scales, gs_out=gs, ws=ws)
+
+        t = _time_graphs(torch, _capture(torch, dev, q), reps)
+        out[f"M{M}_K{K}"] = {"us": round(t * 1e3, 2), "GB/s": round(4.5625 * M * K / (t * 1e-3) / 1e9, 1)}
     return out
 
 

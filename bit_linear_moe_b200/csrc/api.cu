@@ -323,7 +323,7 @@ size_t moe_grouped_linear_workspace(int64_t R, int64_t K, int64_t N, int32_t E, 
     size_t need = 0;
     if (mode == NVFP4_MODE_W4A16) {
         if (epilogue == NVFP4_EPI_COMBINE) need += align256((size_t)(R * N) * 4);
-        need += w4a16_ws(R, K);
+        need += w4a16_ws(R, K) + align256((size_t)E * 4);  // + the touched-expert list
     }
     if (mode == NVFP4_MODE_W4A4) need += grouped_w4a4_ws(nullptr, R, K, N, E, k, epilogue).bytes;
     return need;
@@ -396,6 +396,10 @@ int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const 
     }
     void* xh = wp;
     float* inv = (float*)(wp + align256((size_t)(R * K) * 2));
+    int32_t* touched = (int32_t*)(wp + w4a16_ws(R, K));
+    // at most min(E, R) experts have rows: the grid covers those slots only
+    const int32_t nslots = (int32_t)((int64_t)E < R ? (int64_t)E : R);
+    NVFP4_TRY(launch_touched_experts(expert_offsets, E, nslots, touched, st));
     NVFP4_TRY(launch_x_prep(x, gather ? perm_tok : nullptr, R, K, xh, inv, st));
     GemvArgs a{};
     a.xh = xh;
@@ -410,6 +414,8 @@ int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const 
     a.N = N;
     a.offsets = expert_offsets;
     a.E = E;
+    a.experts = touched;
+    a.n_slots = nslots;
     if (epilogue == NVFP4_EPI_COMBINE) {
         a.epilogue = NVFP4_EPI_NONE;
         a.y = d;

@@ -123,7 +123,8 @@ __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
     const uint8_t* scales = a.scales;
     float gs;
     if (a.offsets) {
-        const int e = blockIdx.x;
+        const int e = a.experts ? a.experts[blockIdx.x] : (int)blockIdx.x;
+        if (e < 0) return;  // slot past the last touched expert (CTA-uniform)
         row_begin = a.offsets[e];
         row_end = a.offsets[e + 1];
         if (row_end <= row_begin) return;  // untouched expert: its weights are never read (CTA-uniform)
@@ -294,7 +295,7 @@ static int launch_cfg(const GemvArgs& a, cudaStream_t st) {
     constexpr int RW = (EPI == NVFP4_EPI_SWIGLU) ? 1 : R;
     const int64_t ncols = (EPI == NVFP4_EPI_SWIGLU) ? a.N / 2 : a.N;
     const int64_t tiles = (ncols + RG * RW - 1) / (RG * RW);
-    const int64_t gx = a.offsets ? a.E : (a.M + MT - 1) / MT;
+    const int64_t gx = a.offsets ? (a.experts ? a.n_slots : a.E) : (a.M + MT - 1) / MT;
     if (tiles > 65535 || gx > 0x7fffffff) return NVFP4_ERR_SHAPE;
     dim3 grid((unsigned)gx, (unsigned)tiles);
     gemv_w4a16_kernel<MT, R, QS, J, LAYOUT, OutT, EPI><<<grid, 256, 0, st>>>(a);
@@ -311,7 +312,13 @@ static int launch_qs(const GemvArgs& a, cudaStream_t st) {
     // target: >= ~8 resident-warp-slots of work per SM (148 SMs x 32 warps)
     int qs = 1;
     while (qs < 8 && warps_at_qs1 * qs < 148 * 48 && nch / (qs * 2) >= 16) qs *= 2;
-    if (a.offsets) qs = nch >= 128 ? 2 : 1;
+    if (a.offsets) {
+        // grouped (decode-time experts, a few rows each): two chunks in flight per
+        // lane keep the register count, and so the resident warps per SM, up
+        qs = nch >= 128 ? 2 : 1;
+        if (qs == 1) return launch_cfg<MT, 2, 1, 2, LAYOUT, OutT, EPI>(a, st);
+        return launch_cfg<MT, 2, 2, 2, LAYOUT, OutT, EPI>(a, st);
+    }
     switch (qs) {
         case 1: return launch_cfg<MT, 2, 1, 6, LAYOUT, OutT, EPI>(a, st);
         case 2: return launch_cfg<MT, 2, 2, 6, LAYOUT, OutT, EPI>(a, st);
@@ -322,7 +329,7 @@ static int launch_qs(const GemvArgs& a, cudaStream_t st) {
 
 template <int LAYOUT, typename OutT, int EPI>
 static int launch_mt(const GemvArgs& a, cudaStream_t st) {
-    const int64_t rows_hint = a.offsets ? 4 : a.M;
+    const int64_t rows_hint = a.offsets ? 2 : a.M;
     if (rows_hint <= 1) return launch_qs<1, LAYOUT, OutT, EPI>(a, st);
     if (rows_hint <= 2) return launch_qs<2, LAYOUT, OutT, EPI>(a, st);
     return launch_qs<4, LAYOUT, OutT, EPI>(a, st);

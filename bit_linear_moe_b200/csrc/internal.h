@@ -41,6 +41,8 @@ struct GemvArgs {
     int64_t N;                // weight rows
     const int32_t* offsets;   // grouped: [E+1] row offsets (nullable for dense)
     int32_t E;
+    const int32_t* experts;   // grouped: touched experts, one per grid slot, -1 = none (nullable: slot = expert)
+    int32_t n_slots;          // grouped: grid slots when `experts` is set
     int epilogue;             // NVFP4_EPI_NONE or NVFP4_EPI_SWIGLU
     void* y;                  // output rows
     int y_dtype;              // NVFP4_DTYPE_F32 / BF16
@@ -87,6 +89,8 @@ int launch_moe_pad(const int32_t* offsets, int32_t E, int64_t rows_pad, const in
                    int32_t* tile_info, int32_t* src_rows, cudaStream_t st);
 int launch_f32_to_bf16(const float* src, int64_t n, void* dst, cudaStream_t st);  // n % 4 == 0
 // tok_of[row_of[i]] = i / k, w_of[row_of[i]] = topk_w[i] for i < n (= T * k).
+// experts with rows, compacted: list[j] for j < nslots (-1 past the last), E <= 1024.
+int launch_touched_experts(const int32_t* offsets, int32_t E, int32_t nslots, int32_t* list, cudaStream_t st);
 int launch_row_token(const int32_t* row_of, const float* topk_w, int64_t n, int32_t k, int32_t* tok_of, float* w_of,
                      cudaStream_t st);
 

@@ -81,8 +81,53 @@ __global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16*
     }
 }
 
+// ---- router logits for a few tokens: one warp per (expert, group of up to 8
+// tokens); the expert's row is streamed once per group, the tokens' rows come
+// from L1/L2 ----
+constexpr int kRouterTokGroup = 8;
+
+__global__ void __launch_bounds__(256) router_logits_small_kernel(const __nv_bfloat16* __restrict__ h,
+                                                                  const __nv_bfloat16* __restrict__ wr,
+                                                                  const float* __restrict__ bias, int64_t T,
+                                                                  int64_t H, int32_t E, float* __restrict__ logits) {
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);  // global warp
+    const int64_t ngroups = (T + kRouterTokGroup - 1) / kRouterTokGroup;
+    if (gw >= (int64_t)E * ngroups) return;
+    const int64_t e = gw / ngroups, t0 = (gw % ngroups) * kRouterTokGroup;
+    const int nt = (int)((T - t0) < kRouterTokGroup ? (T - t0) : kRouterTokGroup);
+    float acc[kRouterTokGroup] = {};
+    for (int64_t k0 = 8 * lane; k0 < H; k0 += 256) {
+        const uint4 wv = ldg_v4(wr + e * H + k0);
+        const uint32_t wu[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int t = 0; t < kRouterTokGroup; ++t) {
+            if (t < nt) {
+                const uint4 hv = ldg_v4(h + (t0 + t) * H + k0);
+                const uint32_t hu[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[t] = fmaf(bf16lo_to_f32(hu[j]), bf16lo_to_f32(wu[j]), acc[t]);
+                    acc[t] = fmaf(bf16hi_to_f32(hu[j]), bf16hi_to_f32(wu[j]), acc[t]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < kRouterTokGroup; ++t) {
+        const float v = warp_sum(acc[t]);
+        if (lane == 0 && t < nt) logits[(t0 + t) * E + e] = v + (bias ? bias[e] : 0.0f);
+    }
+}
+
 int launch_router_logits(const void* h, const void* wr, const float* bias, int64_t T, int64_t H, int32_t E,
                          float* logits, cudaStream_t st) {
+    if (T <= 64 && H % 8 == 0) {
+        const int64_t warps = (int64_t)E * ((T + kRouterTokGroup - 1) / kRouterTokGroup);
+        router_logits_small_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(
+            (const __nv_bfloat16*)h, (const __nv_bfloat16*)wr, bias, T, H, E, logits);
+        return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+    }
     dim3 grid((unsigned)((T + RT - 1) / RT), (unsigned)((E + RT - 1) / RT));
     router_logits_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)h, (const __nv_bfloat16*)wr, bias, T, H, E,
                                                logits);
@@ -373,6 +418,30 @@ int launch_moe_pad(const int32_t* offsets, int32_t E, int64_t rows_pad, const in
 int launch_f32_to_bf16(const float* src, int64_t n, void* dst, cudaStream_t st) {
     const int64_t n4 = n / 4;
     f32_to_bf16_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(src, n4, (__nv_bfloat16*)dst);
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+}
+
+// ---- touched experts: list[j] = the j-th expert with rows, -1 past the last ----
+__global__ void __launch_bounds__(1024) touched_experts_kernel(const int32_t* __restrict__ offsets, int32_t E,
+                                                               int32_t nslots, int32_t* __restrict__ list) {
+    __shared__ int32_t warp_tot[32];
+    const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+    const bool has = e < E && offsets[e + 1] > offsets[e];
+    const uint32_t bal = __ballot_sync(0xffffffffu, has);
+    if (lane == 0) warp_tot[warp] = __popc(bal);
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += warp_tot[w];
+    int total = 0;
+    for (int w = 0; w < 32; ++w) total += warp_tot[w];
+    const int pos = base + __popc(bal & ((1u << lane) - 1u));
+    if (has && pos < nslots) list[pos] = e;
+    for (int j = total + e; j < nslots; j += 1024) list[j] = -1;
+}
+
+int launch_touched_experts(const int32_t* offsets, int32_t E, int32_t nslots, int32_t* list, cudaStream_t st) {
+    if (E < 1 || E > 1024) return NVFP4_ERR_SHAPE;
+    touched_experts_kernel<<<1, 1024, 0, st>>>(offsets, E, nslots, list);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 
