@@ -40,6 +40,7 @@ METRIC = "NVFP4 linear: decode GB/s (% HBM peak); prefill TFLOPS (% FP4 tensor p
 SHAPES = (("qkv", 5120, 10240, 1), ("o_proj", 5120, 5120, 2), ("gate_up", 5120, 34816, 3),
           ("down", 17408, 5120, 4))
 FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
 WORKLOAD = ("dense27b decode linears (QKV 5120x10240, o_proj 5120x5120, gate_up 5120x34816, down 17408x5120), "
             "W4A16, M=1")
 
@@ -198,14 +199,21 @@ def run_native(args, rank, world, dist):
             with torch.cuda.graph(g, stream=side):
                 step(i)
             step_graphs.append(g)
-        for j in range(len(layers)):
-            pair = []
-            for i in range(2):
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=side):
-                    call(j, i)
-                pair.append(g)
-            shape_graphs.append(pair)
+        # one linear alone: each graph launches it once per weight copy, with
+        # enough copies that a replay streams > 3x the L2 (126 MB)
+        for j, (name, K, N, copies, x, y) in enumerate(layers):
+            nc = max(2, -(-3 * L2_BYTES // decode_bytes(1, K, N)))
+            many = [copies[0]] + [tuple(t.clone() for t in copies[0]) for _ in range(nc - 1)]
+
+            def chain(j=j, name=name, many=many, x=x, y=y):
+                for c, s_, g_ in many:
+                    nv.nvfp4_linear(x, c, s_, g_, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16, ws=ws[name])
+
+            chain()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                chain()
+            shape_graphs.append((g, nc, many))
     stream.wait_stream(side)
     torch.cuda.synchronize()
 
@@ -229,23 +237,27 @@ def run_native(args, rank, world, dist):
 
     # per-shape device time: each linear alone, replayed from its graph
     reps = max(200, min(2000, args.steps))
-    per_shape, launch_ms = {}, 0.0
+    per_shape = {}
     for j, (name, K, N, *_) in enumerate(layers):
+        g, nc, _ = shape_graphs[j]
         for i in range(4):
-            shape_graphs[j][i % 2].replay()
+            g.replay()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps_j = max(20, reps // nc)
         a.record(stream)
-        for i in range(reps):
-            shape_graphs[j][i % 2].replay()
+        for i in range(reps_j):
+            g.replay()
         b.record(stream)
         torch.cuda.synchronize()
-        m = a.elapsed_time(b) / reps
-        launch_ms += m
-        per_shape[name] = {"us": round(m * 1e3, 2), "GB/s": round(decode_bytes(1, K, N) / (m * 1e-3) / 1e9, 1)}
+        m = a.elapsed_time(b) / (reps_j * nc)
+        per_shape[name] = {"us": round(m * 1e3, 2), "GB/s": round(decode_bytes(1, K, N) / (m * 1e-3) / 1e9, 1),
+                           "weight_copies": nc}
+    del shape_graphs
 
-    # roofline of the dominant kernel (the W4A16 decode kernel: every launch)
+    # roofline of the dominant kernel: the W4A16 decode kernel is every launch of
+    # the step, so bytes per launch / mean launch time = step bytes / step time
     peak, peak_kind = load_peaks()
-    achieved = step_bytes / (launch_ms * 1e-3) / 1e9
+    achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
     traffic = kernel_traffic("gemv_tma.cu", "gemv_tma_decode")
 
     # end to end through the public API: pinned host x in, host y out, every step
@@ -295,8 +307,8 @@ def run_native(args, rank, world, dist):
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
-                     "per": "decode step (4 launches, one per shape); achieved = algorithmic bytes / summed launch time",
-                     "kernel": "gemv_tma_kernel (the only launch of each linear): per-shape graph replays timed with CUDA events"},
+                     "per": "decode step (4 launches, one per shape): algorithmic bytes / step time on this GPU",
+                     "kernel": "gemv_tma_kernel (the only launch of each linear), CUDA events around the step graphs"},
         "e2e": {"value": round(e2e, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 4 * args.steps,
         "clocks": clk.summary(),
@@ -305,46 +317,49 @@ def run_native(args, rank, world, dist):
     return line
 
 
-def decode_sweep(nv, torch, dev, layers, reps=200):
-    """Per-launch GB/s for each shape and M, from CUDA-graph replays (weights
-    rotated over 2 copies)."""
+def decode_sweep(nv, torch, dev, layers, reps=20):
+    """Per-launch GB/s for each shape and M: a CUDA graph launches the linear once
+    per weight copy, with enough copies that a replay streams > 3x the L2."""
     from bit_linear_moe_b200 import synth
     out = {}
     stream = torch.cuda.current_stream()
     side = torch.cuda.Stream(device=dev)
     for name, K, N, copies, _, _ in layers:
         seed = dict((s[0], s[3]) for s in SHAPES)[name]
+        nc = max(2, -(-3 * L2_BYTES // decode_bytes(1, K, N)))
+        many = [copies[0]] + [tuple(t.clone() for t in copies[0]) for _ in range(nc - 1)]
         row = {}
         for M in synth.DECODE_M:
             x = torch.from_numpy(synth.decode_x(seed, M, K)).to(torch.bfloat16).to(dev)
             y = torch.empty((M, N), dtype=torch.float32, device=dev)
             nbytes = int(nv.lib().nvfp4_linear_workspace(M, K, N, nv.MODE_W4A16))
             ws = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
-            for i in range(3):
-                c, s, g = copies[i % 2]
-                nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16, ws=ws)
+
+            def chain():
+                for c, s, g in many:
+                    nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16, ws=ws)
+
+            chain()
             torch.cuda.synchronize()
             side.wait_stream(stream)
-            graphs = []
             with torch.cuda.stream(side):
-                for i in range(2):
-                    gr = torch.cuda.CUDAGraph()
-                    c, s, g = copies[i]
-                    with torch.cuda.graph(gr, stream=side):
-                        nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16, ws=ws)
-                    graphs.append(gr)
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=side):
+                    chain()
             stream.wait_stream(side)
-            for i in range(4):
-                graphs[i % 2].replay()
+            for i in range(3):
+                gr.replay()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             for i in range(reps):
-                graphs[i % 2].replay()
+                gr.replay()
             b.record(stream)
             torch.cuda.synchronize()
-            m = a.elapsed_time(b) / reps
+            m = a.elapsed_time(b) / (reps * nc)
             row[str(M)] = round(decode_bytes(M, K, N) / (m * 1e-3) / 1e9, 1)
+            del gr
         out[name] = row
+        del many
     return out
 
 

@@ -8,8 +8,9 @@
 //   y[m, n] = gs * sum_q 2^-p_{q,m} * sum_{b in split q} E4M3(s[n, b]) *
 //                                       sum_{k in b} xh_q[m, k] * E2M1(c[n, k])
 //
-// Each CTA stages the bf16 activations of its K split in shared memory, takes
-// their largest magnitude, and rewrites them in place as fp16 scaled by a
+// Each CTA loads the bf16 activations of its K split into shared memory with
+// plain loads (a bulk copy would queue behind the weight stages already
+// requested), takes their largest magnitude, and rewrites them as fp16 scaled by a
 // power of two p that puts that maximum in [2^14, 2^15): exact for every
 // element within 2^28 of the split's maximum.  The split's partial sums are
 // multiplied by 2^-p (exact) before the splits are added.
@@ -27,8 +28,9 @@
 // times; codes are unpacked with cvt.rn.f16x2.e2m1x2 and multiplied with the
 // mixed-precision fma.rn.f32.f16.  The K range of a tile is split over a
 // cluster of QS CTAs (QS chosen so that the grid is one wave over the SMs);
-// their partial sums meet through distributed shared memory and rank 0 writes
-// the output.  Launched as a programmatic dependent: the first ring of weight
+// each CTA stores its partial sums into its own slot of rank 0's shared memory
+// (remote stores, one cluster barrier) and rank 0 adds them and writes the
+// output.  Launched as a programmatic dependent: the first ring of weight
 // stages is requested before the previous kernel in the stream completes, the
 // activations after it.
 #include <cuda.h>
@@ -48,6 +50,7 @@ constexpr int kStageK = 256;                    // elements per stage
 constexpr int kCodeBytes = kTileRows * 128;     // 16 KB
 constexpr int kScaleBytes = 2048;
 constexpr int kThreads = 288;
+constexpr int kMaxQS = 8;                        // K splits per tile (cluster size)
 
 struct DecodeArgs {
     const __nv_bfloat16* x;
@@ -88,7 +91,8 @@ NVFP4_DEV void dot32(const uint4& wq, const uint32_t (&xw)[16], float& p0, float
 }
 
 static size_t decode_smem_bytes(int MT, int64_t kr_max) {
-    return 1024 + (size_t)kStages * (kCodeBytes + kScaleBytes) + (size_t)MT * kr_max * 2 + (size_t)kTileRows * MT * 4 +
+    return 1024 + (size_t)kStages * (kCodeBytes + kScaleBytes) + (size_t)MT * kr_max * 2 +
+           (size_t)kMaxQS * kTileRows * MT * 4 +
            8 * (2 * kStages + 1);
 }
 
@@ -104,11 +108,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint8_t* s_codes = smem;
     uint8_t* s_scales = s_codes + kStages * kCodeBytes;
     __half* s_x = reinterpret_cast<__half*>(s_scales + kStages * kScaleBytes);
-    float* s_red = reinterpret_cast<float*>(s_x + MT * kr_max);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(s_red + kTileRows * MT);
+    float* s_red = reinterpret_cast<float*>(s_x + MT * kr_max);  // [kMaxQS][kTileRows][MT] (rank 0 gathers)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(s_red + kMaxQS * kTileRows * MT);
     uint64_t* full = bars;
     uint64_t* empty = bars + kStages;
-    uint64_t* xbar = bars + 2 * kStages;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = (int)(blockIdx.x % QS);
@@ -125,7 +128,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 8);  // one release per consumer warp
         }
-        mbar_init(xbar, 1);
         fence_barrier_init();
     }
     __syncthreads();
@@ -139,24 +141,17 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int t = 0; t < MT; ++t) inv_p[t] = 1.0f;
 
+    if (QS > 1) cluster_arrive_relaxed();  // waited on before the partial sums are pushed to rank 0
     griddep_launch_dependents();
     if (warp == 8) {
         // ---------------- producer ----------------
         if (lane == 0) {
             prefetch_tensormap(&codes_map);
             if (LAYOUT == NVFP4_SF_ROWMAJOR) prefetch_tensormap(&sc_map);
-            // the first ring's worth of weights goes out before the previous
-            // kernel has finished; the activations only after it
-            const int pre = ns < kStages ? ns : kStages;
+            // weights only: the first ring's worth goes out before the previous
+            // kernel has finished (the consumers fetch the activations)
             for (int s = 0; s < ns; ++s) {
                 const int slot = s % kStages;
-                if (s == pre) {
-                    griddep_wait();
-                    mbar_expect_tx(xbar, (uint32_t)(nt * ns * kStageK * 2));
-                    for (int t = 0; t < nt; ++t)
-                        bulk_load(s_x + t * kr_max, a.x + (m0 + t) * a.K + k_begin, (uint32_t)(ns * kStageK * 2),
-                                  xbar);
-                }
                 if (s >= kStages) {
                     if (!mbar_wait(&empty[slot], ((s / kStages) - 1) & 1, a.status)) break;
                     fence_proxy_async();  // consumers' generic reads before the async-proxy refill
@@ -170,19 +165,16 @@ __global__ void __launch_bounds__(kThreads, 2)
                 else
                     tma_load_2d(s_scales + slot * kScaleBytes, &sc_map, &full[slot], st * 16, (int)row0);
             }
-            if (ns <= kStages) {
-                griddep_wait();
-                mbar_expect_tx(xbar, (uint32_t)(nt * ns * kStageK * 2));
-                for (int t = 0; t < nt; ++t)
-                    bulk_load(s_x + t * kr_max, a.x + (m0 + t) * a.K + k_begin, (uint32_t)(ns * kStageK * 2), xbar);
-            }
         }
+        if (QS > 1) cluster_wait();
     } else {
         griddep_wait();
         // ---------------- consumers ----------------
         const int ch = lane & 7, rsub = lane >> 3;
-        bool ok = mbar_wait(xbar, 0, a.status);
-        // bf16 -> fp16 * 2^p in place, p per token from this split's maximum
+        bool ok = true;
+        // this split's activations, straight from global memory with plain loads
+        // (a bulk copy would queue behind the weight stages already in flight),
+        // then bf16 -> fp16 * 2^p in place, p per token from the split's maximum
         {
             const int ctid = threadIdx.x;  // 0..255 (consumer threads)
             const int nv8 = ns * kStageK / 8;
@@ -190,9 +182,11 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
                 float mx = 0.0f;
-                if (ok && t < nt)
+                if (t < nt)
                     for (int v = ctid; v < nv8; v += 256) {
-                        const uint4 q4 = reinterpret_cast<const uint4*>(s_x + t * kr_max)[v];
+                        const uint4 q4 =
+                            *reinterpret_cast<const uint4*>(a.x + (m0 + t) * a.K + k_begin + (int64_t)v * 8);
+                        reinterpret_cast<uint4*>(s_x + t * kr_max)[v] = q4;
                         const uint32_t u[4] = {q4.x, q4.y, q4.z, q4.w};
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
@@ -213,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 p = p < -126 ? -126 : (p > 126 ? 126 : p);
                 const float sc = __uint_as_float((uint32_t)(127 + p) << 23);
                 inv_p[t] = __uint_as_float((uint32_t)(127 - p) << 23);
-                if (ok && t < nt)
+                if (t < nt)
                     for (int v = ctid; v < nv8; v += 256) {
                         uint4* qp = reinterpret_cast<uint4*>(s_x + t * kr_max) + v;
                         const uint4 q4 = *qp;
@@ -287,13 +281,20 @@ __global__ void __launch_bounds__(kThreads, 2)
                 v += __shfl_xor_sync(0xffffffffu, v, 4);
                 acc[i][t] = v;
             }
+        if (QS > 1) cluster_wait();  // every CTA of the cluster is running: rank 0's memory can be written
         if (ch == 0) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int r = 16 * warp + rsub + 4 * i;
                 if (QS > 1) {
 #pragma unroll
-                    for (int t = 0; t < MT; ++t) s_red[r * MT + t] = acc[i][t] * inv_p[t];
+                    for (int t = 0; t < MT; ++t) {
+                        float* slot = &s_red[((int64_t)q * kTileRows + r) * MT + t];
+                        if (q == 0)
+                            *slot = acc[i][t] * inv_p[t];
+                        else
+                            st_dsmem_f32(slot, 0, acc[i][t] * inv_p[t]);
+                    }
                 } else if (row0 + r < a.N) {
                     const float g = a.gs[0];
 #pragma unroll
@@ -307,18 +308,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 
     if (QS > 1) {
-        cluster_sync();
+        cluster_sync();  // every rank's partial sums are in rank 0's shared memory
         if (q == 0) {
             const float g = a.gs[0];
             for (int idx = threadIdx.x; idx < kTileRows * MT; idx += kThreads) {
                 const int r = idx / MT, t = idx % MT;
                 if (t >= nt || row0 + r >= a.N) continue;
                 float v = s_red[idx];
-                for (int qq = 1; qq < QS; ++qq) v += ld_dsmem_f32(&s_red[idx], (uint32_t)qq);
+                for (int qq = 1; qq < QS; ++qq) v += s_red[(int64_t)qq * kTileRows * MT + idx];
                 store_out<OutT>(reinterpret_cast<OutT*>(a.y) + (m0 + t) * a.ldy + row0 + r, v * g);
             }
         }
-        cluster_sync();
     }
 }
 
@@ -406,8 +406,7 @@ static int run(DecodeArgs a, const uint8_t* codes, const uint8_t* scales, cudaSt
 template <int LAYOUT, typename OutT>
 static int run_mt(const DecodeArgs& a, const uint8_t* codes, const uint8_t* scales, cudaStream_t st) {
     if (a.M <= 1) return run<1, LAYOUT, OutT>(a, codes, scales, st);
-    if (a.M <= 2) return run<2, LAYOUT, OutT>(a, codes, scales, st);
-    return run<4, LAYOUT, OutT>(a, codes, scales, st);
+    return run<2, LAYOUT, OutT>(a, codes, scales, st);
 }
 
 bool decode_tma_supported(int64_t M, int64_t K, int64_t N) {

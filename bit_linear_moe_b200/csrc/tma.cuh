@@ -109,6 +109,15 @@ NVFP4_DEV uint32_t cluster_ctarank() {
 NVFP4_DEV void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+// Split cluster barrier: arrive early (relaxed: orders nothing), wait later.
+NVFP4_DEV void cluster_arrive_relaxed() { asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory"); }
+NVFP4_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+// Store a float to the same shared-memory offset in CTA `rank` of the cluster.
+NVFP4_DEV void st_dsmem_f32(float* local, uint32_t rank, float v) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
+}
 // Read a float from the same shared-memory offset in CTA `rank` of the cluster.
 NVFP4_DEV float ld_dsmem_f32(const float* local, uint32_t rank) {
     uint32_t remote;
