@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // ---------------- producer ----------------
         if (lane == 0) {
             prefetch_tensormap(&codes_map);
+            const uint64_t pol = l2_evict_first_policy();  // weights are read once per call
             if (LAYOUT == NVFP4_SF_ROWMAJOR) prefetch_tensormap(&sc_map);
             // weights only: the first ring's worth goes out before the previous
             // kernel has finished (the consumers fetch the activations)
@@ -158,12 +159,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
                 mbar_expect_tx(&full[slot], kCodeBytes + kScaleBytes);
                 const int st = st_begin + s;
-                tma_load_2d(s_codes + slot * kCodeBytes, &codes_map, &full[slot], st * 128, (int)row0);
+                tma_load_2d_hint(s_codes + slot * kCodeBytes, &codes_map, &full[slot], st * 128, (int)row0, pol);
                 if (LAYOUT == NVFP4_SF_TILED)
-                    bulk_load(s_scales + slot * kScaleBytes, a.scales + ((int64_t)tile * a.cp4 + (int64_t)st * 4) * 512,
-                              kScaleBytes, &full[slot]);
+                    bulk_load_hint(s_scales + slot * kScaleBytes,
+                                   a.scales + ((int64_t)tile * a.cp4 + (int64_t)st * 4) * 512, kScaleBytes, &full[slot],
+                                   pol);
                 else
-                    tma_load_2d(s_scales + slot * kScaleBytes, &sc_map, &full[slot], st * 16, (int)row0);
+                    tma_load_2d_hint(s_scales + slot * kScaleBytes, &sc_map, &full[slot], st * 16, (int)row0, pol);
             }
         }
         if (QS > 1) cluster_wait();
@@ -179,22 +181,39 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int ctid = threadIdx.x;  // 0..255 (consumer threads)
             const int nv8 = ns * kStageK / 8;
             float* s_max = s_red;          // reused before the reduction needs it
+            // every load of a thread is in flight before the first is used
+            float mx[MT];
 #pragma unroll
-            for (int t = 0; t < MT; ++t) {
-                float mx = 0.0f;
-                if (t < nt)
-                    for (int v = ctid; v < nv8; v += 256) {
-                        const uint4 q4 =
-                            *reinterpret_cast<const uint4*>(a.x + (m0 + t) * a.K + k_begin + (int64_t)v * 8);
-                        reinterpret_cast<uint4*>(s_x + t * kr_max)[v] = q4;
-                        const uint32_t u[4] = {q4.x, q4.y, q4.z, q4.w};
+            for (int t = 0; t < MT; ++t) mx[t] = 0.0f;
+            for (int base = ctid; base < nv8; base += 4 * 256) {
+                uint4 q4[MT][4];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            mx = fmaxf(mx, fmaxf(fabsf(bf16lo_to_f32(u[j])), fabsf(bf16hi_to_f32(u[j]))));
+                for (int t = 0; t < MT; ++t)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int v = base + i * 256;
+                        if (t < nt && v < nv8)
+                            q4[t][i] = *reinterpret_cast<const uint4*>(a.x + (m0 + t) * a.K + k_begin + (int64_t)v * 8);
                     }
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                if (lane == 0) s_max[t * 8 + warp] = mx;
+                for (int t = 0; t < MT; ++t)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int v = base + i * 256;
+                        if (t < nt && v < nv8) {
+                            reinterpret_cast<uint4*>(s_x + t * kr_max)[v] = q4[t][i];
+                            const uint32_t u[4] = {q4[t][i].x, q4[t][i].y, q4[t][i].z, q4[t][i].w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                mx[t] = fmaxf(mx[t], fmaxf(fabsf(bf16lo_to_f32(u[j])), fabsf(bf16hi_to_f32(u[j]))));
+                        }
+                    }
+            }
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) mx[t] = fmaxf(mx[t], __shfl_xor_sync(0xffffffffu, mx[t], o));
+                if (lane == 0) s_max[t * 8 + warp] = mx[t];
             }
             asm volatile("bar.sync 1, 256;" ::: "memory");
 #pragma unroll

@@ -62,7 +62,8 @@ def test_dense27b_decode(name, K, N, seed, M):
 
 
 @pytest.mark.parametrize("M,K,N", [(1, 16, 1), (3, 48, 3), (5, 80, 130), (2, 4096, 257), (7, 1040, 1000),
-                                   (33, 256, 64), (1, 17408, 8), (4, 32, 2048)])
+                                   (33, 256, 64), (1, 17408, 8), (4, 32, 2048), (1, 256, 19277), (2, 512, 37000),
+                                   (1, 256, 40000), (2, 512, 60000)])
 @pytest.mark.parametrize("layout", [nv.SF_ROWMAJOR, nv.SF_TILED])
 def test_ragged(M, K, N, layout):
     rng = np.random.default_rng(M * 1000 + K + N)
