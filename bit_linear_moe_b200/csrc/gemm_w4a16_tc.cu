@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(w4a16tc::kThreads, 1)
         if (lane == 0) {
             prefetch_tensormap(&map_w);
             prefetch_tensormap(&map_x);
+            const uint64_t pol = l2_evict_first_policy();  // weights are read once per call
             const uint8_t* sf_tile = a.scales + (int64_t)tile * cp4 * 512;
             for (int s = 0; s < ns; ++s) {
                 const int slot = s % kStages;
@@ -135,11 +136,11 @@ __global__ void __launch_bounds__(w4a16tc::kThreads, 1)
                 uint8_t* st = smem + slot * C::kStageBytes;
                 const int kst = st_begin + s;
                 mbar_expect_tx(&full[slot], C::kStageBytes);
-                tma_load_2d(st, &map_w, &full[slot], kst * 128, (int)row0);
+                tma_load_2d_hint(st, &map_w, &full[slot], kst * 128, (int)row0, pol);
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
                     tma_load_2d(st + kCodes + c * NT * 128, &map_x, &full[slot], kst * 512 + c * 128, 0);
-                bulk_load(st + kCodes + C::kX, sf_tile + (int64_t)kst * 4 * 512, kSf, &full[slot]);
+                bulk_load_hint(st + kCodes + C::kX, sf_tile + (int64_t)kst * 4 * 512, kSf, &full[slot], pol);
             }
         }
     } else if (warp == 1) {
