@@ -14,7 +14,7 @@ __device__ int g_device_status = 0;
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 // Device address of the status word, looked up once per device.
-static int* device_status_ptr() {
+int* device_status_ptr() {
     static int* cache[64] = {nullptr};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;

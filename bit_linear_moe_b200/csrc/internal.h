@@ -72,6 +72,12 @@ int launch_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales, const floa
                      int y_dtype, int* status, cudaStream_t st);
 
 // moe.cu
+// router_tc.cu: tensor-core router logits (T > 64, H % 64 == 0, 16-byte aligned rows)
+bool router_tc_supported(const void* h, const void* wr, int64_t T, int64_t H, int32_t E);
+int launch_router_logits_tc(const void* h, const void* wr, const float* bias, int64_t T, int64_t H, int32_t E,
+                            float* logits, int* status, cudaStream_t st);
+// Device address of the library's status word (timeouts of bounded waits).
+int* device_status_ptr();
 int launch_router_logits(const void* h, const void* wr, const float* bias, int64_t T, int64_t H, int32_t E,
                          float* logits, cudaStream_t st);
 int launch_topk_count(const float* logits, int64_t T, int32_t E, int32_t k, int32_t* topk_idx, float* topk_w,

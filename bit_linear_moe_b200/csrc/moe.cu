@@ -128,6 +128,8 @@ int launch_router_logits(const void* h, const void* wr, const float* bias, int64
             (const __nv_bfloat16*)h, (const __nv_bfloat16*)wr, bias, T, H, E, logits);
         return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
     }
+    if (router_tc_supported(h, wr, T, H, E))
+        return launch_router_logits_tc(h, wr, bias, T, H, E, logits, device_status_ptr(), st);
     dim3 grid((unsigned)((T + RT - 1) / RT), (unsigned)((E + RT - 1) / RT));
     router_logits_kernel<<<grid, 256, 0, st>>>((const __nv_bfloat16*)h, (const __nv_bfloat16*)wr, bias, T, H, E,
                                                logits);

@@ -74,6 +74,41 @@ def test_route_ties_go_to_lower_index():
     assert np.allclose(out["topk_w"].cpu().numpy()[:, :5], np.exp(0.5) / (5 * np.exp(0.5) + np.exp(0.25)))
 
 
+@pytest.mark.parametrize("T,Hs,Es,with_bias", [(300, 128, 96, True), (129, 1088, 90, False), (65, 64, 512, True),
+                                                (1000, 2048, 130, True)])
+def test_router_tensor_core_shapes(T, Hs, Es, with_bias):
+    """Token counts above 64 run the tensor-core router: ragged token and
+    expert tiles, a K ring that wraps, expert counts that are not a multiple
+    of 4 (scalar stores)."""
+    rng = np.random.default_rng(T + Hs + Es)
+    h = synth.to_bf16(rng.standard_normal((T, Hs)).astype(np.float32))
+    wr = synth.to_bf16((0.05 * rng.standard_normal((Es, Hs))).astype(np.float32))
+    bias = (0.1 * rng.standard_normal(Es)).astype(np.float32) if with_bias else None
+    k = 6
+    out = nv.moe_route_topk(torch.from_numpy(h).to(torch.bfloat16).cuda(), torch.from_numpy(wr).to(torch.bfloat16).cuda(),
+                            k, logit_bias=None if bias is None else torch.from_numpy(bias).cuda(), want_logits=True)
+    torch.cuda.synchronize()
+    g = {n: v.cpu().numpy() for n, v in out.items()}
+    ref = omoe.router_logits(h, wr, bias)
+    absdot = np.abs(h.astype(np.float64)) @ np.abs(wr.astype(np.float64)).T
+    assert_within_bound(g["logits"], ref, absdot, False, f"router logits T={T} H={Hs} E={Es}")
+    idx, _ = omoe.topk(g["logits"].astype(np.float64), k)
+    assert np.array_equal(g["topk_idx"], idx)
+
+
+def test_route_ties_go_to_lower_index_tensor_core():
+    T, Hs, Es = 100, 64, 40
+    h = np.zeros((T, Hs), np.float32)
+    h[:, 0] = 1.0
+    wr = np.zeros((Es, Hs), np.float32)
+    wr[[3, 7, 11, 20, 33], 0] = 0.5
+    wr[[1, 2], 0] = 0.25
+    out = nv.moe_route_topk(torch.from_numpy(h).to(torch.bfloat16).cuda(),
+                            torch.from_numpy(wr).to(torch.bfloat16).cuda(), 6, want_logits=True)
+    idx = out["topk_idx"].cpu().numpy()
+    assert (idx == np.array([3, 7, 11, 20, 33, 1])).all()
+
+
 class _Experts:
     """Expert weights for the routed-expert tests.  The oracle quantizes every
     expert it checks; untouched experts hold zeros (they are never read)."""
