@@ -137,48 +137,64 @@ int launch_router_logits(const void* h, const void* wr, const float* bias, int64
 }
 
 // ---- top-k + per-block expert counts ------------------------------------
-// CTA = 256 threads = 8 warps, kPermBlockTokens tokens; a warp takes 16 tokens.
-constexpr int kMaxE = 1024, kMaxPerLane = kMaxE / 32;
+// CTA = 1024 threads = 32 warps, kPermBlockTokens tokens; a warp takes 4
+// tokens.  Lane l holds logits l, l + 32, ... (PER of them) and keeps the best
+// of its untaken ones; a round is a warp arg-max over the lanes' bests, after
+// which only the winning lane rescans its own values.
+constexpr int kMaxE = 1024, kTopkThreads = 1024;
 
 NVFP4_DEV bool better(float v, int i, float bv, int bi) { return v > bv || (v == bv && i < bi); }
 
-__global__ void __launch_bounds__(256) topk_count_kernel(const float* __restrict__ logits, int64_t T, int32_t E,
-                                                         int32_t k, int32_t* __restrict__ topk_idx,
-                                                         float* __restrict__ topk_w,
-                                                         int32_t* __restrict__ blk_counts) {
+template <int PER>
+__global__ void __launch_bounds__(kTopkThreads) topk_count_kernel(const float* __restrict__ logits, int64_t T,
+                                                                  int32_t E, int32_t k, int32_t* __restrict__ topk_idx,
+                                                                  float* __restrict__ topk_w,
+                                                                  int32_t* __restrict__ blk_counts) {
     __shared__ uint32_t mask[kMaxE][kPermBlockTokens / 32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < E * (kPermBlockTokens / 32); i += blockDim.x) (&mask[0][0])[i] = 0;
     __syncthreads();
     const int64_t tb = (int64_t)blockIdx.x * kPermBlockTokens;
-    const int per_lane = (E + 31) / 32;
-    for (int tt = warp; tt < kPermBlockTokens; tt += 8) {
+    for (int tt = warp; tt < kPermBlockTokens; tt += kTopkThreads / 32) {
         const int64_t t = tb + tt;
         if (t >= T) break;
-        float v[kMaxPerLane];
+        float v[PER];
 #pragma unroll
-        for (int i = 0; i < kMaxPerLane; ++i) {
+        for (int i = 0; i < PER; ++i) {
             const int e = i * 32 + lane;
-            v[i] = (i < per_lane && e < E) ? logits[t * E + e] : -INFINITY;
+            v[i] = e < E ? logits[t * E + e] : -INFINITY;
         }
         uint32_t taken = 0;  // bit i: v[i] already selected
+        auto rescan = [&](float& lbv, int& lbi) {
+            lbv = -INFINITY;
+            lbi = 0x7fffffff;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int e = i * 32 + lane;
+                if (e < E && !((taken >> i) & 1u) && better(v[i], e, lbv, lbi)) {
+                    lbv = v[i];
+                    lbi = e;
+                }
+            }
+        };
+        float lbv;
+        int lbi;
+        rescan(lbv, lbi);
         float lmax = 0.0f, mywl = 0.0f;
         int myidx = 0;
         for (int j = 0; j < k; ++j) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-#pragma unroll
-            for (int i = 0; i < kMaxPerLane; ++i) {
-                const int e = i * 32 + lane;
-                if (i < per_lane && e < E && !((taken >> i) & 1u) && better(v[i], e, bv, bi)) { bv = v[i]; bi = e; }
-            }
+            float bv = lbv;
+            int bi = lbi;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
                 const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
                 if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
             }
-            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+            if ((bi & 31) == lane) {
+                taken |= 1u << (bi >> 5);
+                rescan(lbv, lbi);
+            }
             if (j == 0) lmax = bv;
             if (lane == j) { myidx = bi; mywl = bv; }
         }
@@ -202,7 +218,13 @@ __global__ void __launch_bounds__(256) topk_count_kernel(const float* __restrict
 int launch_topk_count(const float* logits, int64_t T, int32_t E, int32_t k, int32_t* topk_idx, float* topk_w,
                       int32_t* blk_counts, cudaStream_t st) {
     const int64_t nblk = (T + kPermBlockTokens - 1) / kPermBlockTokens;
-    topk_count_kernel<<<(unsigned)nblk, 256, 0, st>>>(logits, T, E, k, topk_idx, topk_w, blk_counts);
+    const int per = (E + 31) / 32;
+    if (per <= 8)
+        topk_count_kernel<8><<<(unsigned)nblk, kTopkThreads, 0, st>>>(logits, T, E, k, topk_idx, topk_w, blk_counts);
+    else if (per <= 16)
+        topk_count_kernel<16><<<(unsigned)nblk, kTopkThreads, 0, st>>>(logits, T, E, k, topk_idx, topk_w, blk_counts);
+    else
+        topk_count_kernel<32><<<(unsigned)nblk, kTopkThreads, 0, st>>>(logits, T, E, k, topk_idx, topk_w, blk_counts);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 

@@ -75,7 +75,7 @@ def test_route_ties_go_to_lower_index():
 
 
 @pytest.mark.parametrize("T,Hs,Es,with_bias", [(300, 128, 96, True), (129, 1088, 90, False), (65, 64, 512, True),
-                                                (1000, 2048, 130, True)])
+                                                (1000, 2048, 130, True), (200, 128, 700, False)])
 def test_router_tensor_core_shapes(T, Hs, Es, with_bias):
     """Token counts above 64 run the tensor-core router: ragged token and
     expert tiles, a K ring that wraps, expert counts that are not a multiple
