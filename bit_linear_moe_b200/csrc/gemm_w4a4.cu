@@ -183,13 +183,34 @@ __global__ void __launch_bounds__(w4a4::kThreads, 1)
             if (ok) tc_commit(accum);
         }
     } else {
-        // epilogue: warps 2..5 -> tensor-memory lane quadrants 2, 3, 0, 1
+        // epilogue: warps 2..5 -> tensor-memory lane quadrants 2, 3, 0, 1.  The
+        // whole accumulator row goes to registers first; then warp 0 frees the
+        // tensor memory while the stores run.
         const int q = warp & 3;
         const bool ok = mbar_wait(accum, 0, a.status);
         tc_fence_after();
         const int i = 32 * q + lane;  // row within the tile
         const bool row_ok = ok && i < nvalid;
         const float g = ok ? a.gs_a[0] * a.gs_b[GROUPED ? expert : 0] : 0.0f;
+        uint32_t r[BN / 32][32];
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c) {
+            tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + 32 * c, r[c]);
+            if constexpr (EPI == NVFP4_EPI_SWIGLU) {
+                uint32_t u[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + 128 + 32 * c, u);
+                tmem_ld_wait();
+#pragma unroll
+                for (int t = 0; t < 32; ++t)
+                    r[c][t] = __float_as_uint(silu(__uint_as_float(r[c][t]) * g) * (__uint_as_float(u[t]) * g));
+            } else {
+                tmem_ld_wait();
+#pragma unroll
+                for (int t = 0; t < 32; ++t) r[c][t] = __float_as_uint(__uint_as_float(r[c][t]) * g);
+            }
+        }
+        tc_fence_before();
+        asm volatile("bar.arrive 2, 160;" ::: "memory");  // warps 2-5 done with tensor memory
         const int64_t orow = out_row0 + i;
         int64_t tok = 0;
         float wgt = 0.0f;
@@ -200,35 +221,22 @@ __global__ void __launch_bounds__(w4a4::kThreads, 1)
             }
         }
         const int64_t ncols = (EPI == NVFP4_EPI_SWIGLU) ? a.N / 2 : a.N;
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + c0, r);
-            if constexpr (EPI == NVFP4_EPI_SWIGLU) {
-                uint32_t u[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + 128 + c0, u);
-                tmem_ld_wait();
 #pragma unroll
-                for (int t = 0; t < 32; ++t)
-                    r[t] = __float_as_uint(silu(__uint_as_float(r[t]) * g) * (__uint_as_float(u[t]) * g));
-            } else {
-                tmem_ld_wait();
-#pragma unroll
-                for (int t = 0; t < 32; ++t) r[t] = __float_as_uint(__uint_as_float(r[t]) * g);
-            }
+        for (int c = 0; c < BN / 32; ++c) {
             if (!row_ok) continue;
-            const int64_t col = col0 + c0;
+            const int64_t col = col0 + 32 * c;
             if constexpr (EPI == NVFP4_EPI_COMBINE) {
                 float* yr = a.yacc + tok * a.ldy + col;
                 if (col + 32 <= ncols && (a.ldy & 3) == 0) {
 #pragma unroll
                     for (int t = 0; t < 32; t += 4)
                         asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(yr + t),
-                                     "f"(wgt * __uint_as_float(r[t])), "f"(wgt * __uint_as_float(r[t + 1])),
-                                     "f"(wgt * __uint_as_float(r[t + 2])), "f"(wgt * __uint_as_float(r[t + 3]))
+                                     "f"(wgt * __uint_as_float(r[c][t])), "f"(wgt * __uint_as_float(r[c][t + 1])),
+                                     "f"(wgt * __uint_as_float(r[c][t + 2])), "f"(wgt * __uint_as_float(r[c][t + 3]))
                                      : "memory");
                 } else {
                     for (int t = 0; t < 32; ++t)
-                        if (col + t < ncols) atomicAdd(yr + t, wgt * __uint_as_float(r[t]));
+                        if (col + t < ncols) atomicAdd(yr + t, wgt * __uint_as_float(r[c][t]));
                 }
             } else {
                 OutT* yrow = reinterpret_cast<OutT*>(a.y) + orow * a.ldy;
@@ -237,16 +245,16 @@ __global__ void __launch_bounds__(w4a4::kThreads, 1)
 #pragma unroll
                         for (int t = 0; t < 32; t += 4)
                             *reinterpret_cast<float4*>(yrow + col + t) =
-                                make_float4(__uint_as_float(r[t]), __uint_as_float(r[t + 1]),
-                                            __uint_as_float(r[t + 2]), __uint_as_float(r[t + 3]));
+                                make_float4(__uint_as_float(r[c][t]), __uint_as_float(r[c][t + 1]),
+                                            __uint_as_float(r[c][t + 2]), __uint_as_float(r[c][t + 3]));
                     } else {
 #pragma unroll
                         for (int t = 0; t < 32; t += 8) {
                             uint32_t w[4];
 #pragma unroll
                             for (int u2 = 0; u2 < 4; ++u2) {
-                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[t + 2 * u2]),
-                                                                                __uint_as_float(r[t + 2 * u2 + 1]));
+                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[c][t + 2 * u2]),
+                                                                                __uint_as_float(r[c][t + 2 * u2 + 1]));
                                 w[u2] = *reinterpret_cast<const uint32_t*>(&b2);
                             }
                             *reinterpret_cast<uint4*>(yrow + col + t) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -254,14 +262,14 @@ __global__ void __launch_bounds__(w4a4::kThreads, 1)
                     }
                 } else {
                     for (int t = 0; t < 32; ++t)
-                        if (col + t < ncols) store_out<OutT>(yrow + col + t, __uint_as_float(r[t]));
+                        if (col + t < ncols) store_out<OutT>(yrow + col + t, __uint_as_float(r[c][t]));
                 }
             }
         }
     }
-    tc_fence_before();
-    __syncthreads();
     if (warp == 0) {
+        // every MMA completed before the epilogue read the accumulator
+        asm volatile("bar.sync 2, 160;" ::: "memory");
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
