@@ -47,6 +47,7 @@ constexpr int BM = 128, BN = 128, BK = 256;  // BK elements = 128 bytes per row
 constexpr int kStages = 3;
 constexpr int kTile = 128 * 128, kSf = 2048;
 constexpr int kThreads = 192;
+constexpr int kOutStride = BN + 4;  // staged output row, floats (16-byte rows, conflict-free float4 stores)
 template <int NB>
 struct Cfg {
     static constexpr int kStageBytes = kTile * (1 + NB) + kSf * (1 + NB);
@@ -72,7 +73,10 @@ struct GemmArgs {
     int* status;
 };
 
-NVFP4_DEV float silu(float g) { return g / (1.0f + expf(-g)); }
+// silu(g) = g * sigmoid(g) with the hardware exponential and divide (a few
+// ulp; the IEEE-rounded expf and division cost 10x more here, where one warp
+// per scheduler runs the epilogue and nothing hides their latency).
+NVFP4_DEV float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 template <typename OutT, int EPI, bool GROUPED>
 __global__ void __launch_bounds__(w4a4::kThreads, 1)
@@ -190,7 +194,6 @@ __global__ void __launch_bounds__(w4a4::kThreads, 1)
         const bool ok = mbar_wait(accum, 0, a.status);
         tc_fence_after();
         const int i = 32 * q + lane;  // row within the tile
-        const bool row_ok = ok && i < nvalid;
         const float g = ok ? a.gs_a[0] * a.gs_b[GROUPED ? expert : 0] : 0.0f;
         uint32_t r[BN / 32][32];
 #pragma unroll
@@ -211,58 +214,51 @@ __global__ void __launch_bounds__(w4a4::kThreads, 1)
         }
         tc_fence_before();
         asm volatile("bar.arrive 2, 160;" ::: "memory");  // warps 2-5 done with tensor memory
-        const int64_t orow = out_row0 + i;
-        int64_t tok = 0;
-        float wgt = 0.0f;
-        if constexpr (EPI == NVFP4_EPI_COMBINE) {
-            if (row_ok) {
-                tok = a.tok_of[orow];
-                wgt = a.w_of[orow];
-            }
-        }
+        // Stage the tile in shared memory (the ring is idle: every MMA that read
+        // it has completed), then write it out row by row so that a warp's
+        // stores (or reductions) cover contiguous runs of one output row.
+        float* so = reinterpret_cast<float*>(smem);  // [BM][kOutStride]
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+            for (int t = 0; t < 32; t += 4)
+                *reinterpret_cast<float4*>(so + i * kOutStride + 32 * c + t) =
+                    make_float4(__uint_as_float(r[c][t]), __uint_as_float(r[c][t + 1]), __uint_as_float(r[c][t + 2]),
+                                __uint_as_float(r[c][t + 3]));
+        asm volatile("bar.sync 3, 128;" ::: "memory");
         const int64_t ncols = (EPI == NVFP4_EPI_SWIGLU) ? a.N / 2 : a.N;
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-            if (!row_ok) continue;
-            const int64_t col = col0 + 32 * c;
+        const int64_t col = col0 + 4 * lane;  // this lane's 4 columns
+        const int nrows = ok ? nvalid : 0;
+        for (int rr = warp - 2; rr < nrows; rr += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(so + rr * kOutStride + 4 * lane);
+            const float vv[4] = {v.x, v.y, v.z, v.w};
+            const int64_t orow = out_row0 + rr;
             if constexpr (EPI == NVFP4_EPI_COMBINE) {
+                const int64_t tok = a.tok_of[orow];
+                const float wgt = a.w_of[orow];
                 float* yr = a.yacc + tok * a.ldy + col;
-                if (col + 32 <= ncols && (a.ldy & 3) == 0) {
-#pragma unroll
-                    for (int t = 0; t < 32; t += 4)
-                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(yr + t),
-                                     "f"(wgt * __uint_as_float(r[c][t])), "f"(wgt * __uint_as_float(r[c][t + 1])),
-                                     "f"(wgt * __uint_as_float(r[c][t + 2])), "f"(wgt * __uint_as_float(r[c][t + 3]))
-                                     : "memory");
+                if (col + 4 <= ncols && (a.ldy & 3) == 0) {
+                    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(yr), "f"(wgt * v.x),
+                                 "f"(wgt * v.y), "f"(wgt * v.z), "f"(wgt * v.w)
+                                 : "memory");
                 } else {
-                    for (int t = 0; t < 32; ++t)
-                        if (col + t < ncols) atomicAdd(yr + t, wgt * __uint_as_float(r[c][t]));
+                    for (int t = 0; t < 4; ++t)
+                        if (col + t < ncols) atomicAdd(yr + t, wgt * vv[t]);
                 }
             } else {
-                OutT* yrow = reinterpret_cast<OutT*>(a.y) + orow * a.ldy;
-                if (col + 32 <= ncols && (a.ldy & 7) == 0) {
+                OutT* yp = reinterpret_cast<OutT*>(a.y) + orow * a.ldy + col;
+                if (col + 4 <= ncols && (a.ldy & 3) == 0) {
                     if constexpr (sizeof(OutT) == 4) {
-#pragma unroll
-                        for (int t = 0; t < 32; t += 4)
-                            *reinterpret_cast<float4*>(yrow + col + t) =
-                                make_float4(__uint_as_float(r[c][t]), __uint_as_float(r[c][t + 1]),
-                                            __uint_as_float(r[c][t + 2]), __uint_as_float(r[c][t + 3]));
+                        *reinterpret_cast<float4*>(yp) = v;
                     } else {
-#pragma unroll
-                        for (int t = 0; t < 32; t += 8) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int u2 = 0; u2 < 4; ++u2) {
-                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[c][t + 2 * u2]),
-                                                                                __uint_as_float(r[c][t + 2 * u2 + 1]));
-                                w[u2] = *reinterpret_cast<const uint32_t*>(&b2);
-                            }
-                            *reinterpret_cast<uint4*>(yrow + col + t) = make_uint4(w[0], w[1], w[2], w[3]);
-                        }
+                        const __nv_bfloat162 b0 = __floats2bfloat162_rn(v.x, v.y);
+                        const __nv_bfloat162 b1 = __floats2bfloat162_rn(v.z, v.w);
+                        *reinterpret_cast<uint2*>(yp) =
+                            make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
                     }
                 } else {
-                    for (int t = 0; t < 32; ++t)
-                        if (col + t < ncols) store_out<OutT>(yrow + col + t, __uint_as_float(r[c][t]));
+                    for (int t = 0; t < 4; ++t)
+                        if (col + t < ncols) store_out<OutT>(yp + t, vv[t]);
                 }
             }
         }
