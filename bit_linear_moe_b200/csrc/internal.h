@@ -107,6 +107,8 @@ int launch_gemm_w4a4_grouped(const uint8_t* a_codes, const uint8_t* a_scales, co
                              int y_dtype, float* yacc, const int32_t* tok_of, const float* w_of, int* status,
                              cudaStream_t st);
 
-constexpr int kPermBlockTokens = 128;
+// Tokens per block of the routing permutation (top-k, counts, scatter): 32
+// gives one CTA per 32 tokens, so a 4,096-token batch spreads over 128 SMs.
+constexpr int kPermBlockTokens = 32;
 
 }  // namespace nvfp4

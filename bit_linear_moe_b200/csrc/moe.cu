@@ -9,7 +9,7 @@
 //                (logit descending, expert index ascending); weights are the
 //                softmax over the k winners.
 // Permutation    counting sort by expert, stable in token order, without
-//                atomics on the result: per block of 128 tokens a bitmask per
+//                atomics on the result: per block of 32 tokens a bitmask per
 //                expert marks the tokens that chose it, so a token's rank inside
 //                its block is a popcount; block bases come from a scan.
 // Combine        y[t, n] = sum_j w[t, j] * d[row_of[t, j], n], j ascending.
@@ -137,8 +137,8 @@ int launch_router_logits(const void* h, const void* wr, const float* bias, int64
 }
 
 // ---- top-k + per-block expert counts ------------------------------------
-// CTA = 1024 threads = 32 warps, kPermBlockTokens tokens; a warp takes 4
-// tokens.  Lane l holds logits l, l + 32, ... (PER of them) and keeps the best
+// CTA = 1024 threads = 32 warps, kPermBlockTokens tokens; a warp takes
+// kPermBlockTokens / 32 of them.  Lane l holds logits l, l + 32, ... (PER of them) and keeps the best
 // of its untaken ones; a round is a warp arg-max over the lanes' bests, after
 // which only the winning lane rescans its own values.
 constexpr int kMaxE = 1024, kTopkThreads = 1024;
@@ -234,13 +234,16 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(const int32_t* __restri
                                                          int32_t* __restrict__ blk_base) {
     __shared__ int32_t tot[kMaxE];
     const int e = threadIdx.x;
+    constexpr int kU = 8;  // counts loaded per round trip
     int32_t run = 0;
-    if (e < E) {
-        for (int64_t b = 0; b < nblk; ++b) {
-            blk_base[b * E + e] = run;
-            run += blk_counts[b * E + e];
+    if (e < E)
+        for (int64_t b0 = 0; b0 < nblk; b0 += kU) {
+            int32_t c[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) c[u] = b0 + u < nblk ? blk_counts[(b0 + u) * E + e] : 0;
+#pragma unroll
+            for (int u = 0; u < kU; ++u) run += c[u];
         }
-    }
     tot[e] = e < E ? run : 0;
     __syncthreads();
     // Hillis-Steele inclusive scan over 1024 entries.
@@ -254,7 +257,18 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(const int32_t* __restri
         const int32_t excl = tot[e] - run;
         offsets[e] = excl;
         if (e == E - 1) offsets[E] = tot[e];
-        for (int64_t b = 0; b < nblk; ++b) blk_base[b * E + e] += excl;
+        int32_t base = excl;
+        for (int64_t b0 = 0; b0 < nblk; b0 += kU) {
+            int32_t c[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) c[u] = b0 + u < nblk ? blk_counts[(b0 + u) * E + e] : 0;
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+                if (b0 + u < nblk) {
+                    blk_base[(b0 + u) * E + e] = base;
+                    base += c[u];
+                }
+        }
     }
 }
 

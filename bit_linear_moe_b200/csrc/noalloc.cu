@@ -8,7 +8,7 @@
 // outputs as moe_route_topk but no workspace: its scratch is the file-scope
 // array below, which every GPU that loads the library holds until exit.
 //
-// The scratch holds the per-128-token-block expert counts and bases and, when
+// The scratch holds the per-32-token-block expert counts and bases and, when
 // the caller passes no logits buffer, the logits.  Every byte the kernels read
 // from it they first write in the same call, so nothing needs clearing.  All
 // calls share the one array: calls that overlap on the GPU (other streams,

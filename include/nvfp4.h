@@ -203,7 +203,7 @@ int moe_route_topk(const void* h, const void* w_router, const float* logit_bias,
  * must not grow inside a step, or code where an allocation would stall the
  * device or is not permitted), so it takes no workspace.  Its scratch is a
  * 1 MiB array inside the library that every GPU loading the library holds
- * until exit.  It needs ceil(T/128) * E * 8 bytes (rounded up to 256-byte
+ * until exit.  It needs ceil(T/32) * E * 8 bytes (rounded up to 256-byte
  * pieces), plus T * E * 4 bytes when logits_out is NULL; a request that does
  * not fit returns NVFP4_ERR_WORKSPACE before launching anything (pass
  * logits_out to route large T).  The first call on a device looks up the
