@@ -21,7 +21,10 @@
 //            32x128b.warpx4) and issues 4 MMAs of K = 64 per B tile and stage,
 //            then commits to the stage's empty barrier;
 //   warps 2-5 wait for the last commit, read the fp32 accumulators with
-//            tcgen05.ld (each warp its 32-lane quadrant) and run the epilogue.
+//            tcgen05.ld (each warp its 32-lane quadrant) into registers and
+//            apply the epilogue; warp 0 then frees the tensor memory while
+//            they stage the tile in the idle ring's shared memory and write
+//            it out one contiguous output-row run per warp instruction.
 //
 // Grouped form (mixture of experts; CHImp Alpha v1.0 model card, "How it fits
 // on one GPU"): the permuted activations are laid out with each expert's rows
