@@ -329,7 +329,10 @@ static int launch_qs(const GemvArgs& a, cudaStream_t st) {
 
 template <int LAYOUT, typename OutT, int EPI>
 static int launch_mt(const GemvArgs& a, cudaStream_t st) {
-    const int64_t rows_hint = a.offsets ? 2 : a.M;
+    // grouped: most touched experts hold one or two rows at decode sizes; one
+    // activation row per pass halves the activation reads for a single-row
+    // expert (experts with more rows take more passes over their weights)
+    const int64_t rows_hint = a.offsets ? (a.M <= 2 * (int64_t)a.n_slots ? 1 : 2) : a.M;
     if (rows_hint <= 1) return launch_qs<1, LAYOUT, OutT, EPI>(a, st);
     if (rows_hint <= 2) return launch_qs<2, LAYOUT, OutT, EPI>(a, st);
     return launch_qs<4, LAYOUT, OutT, EPI>(a, st);
