@@ -24,7 +24,8 @@
 // on one GPU": only the chosen experts are read): grid.x walks the experts,
 // expert e's rows are [offsets[e], offsets[e+1]); an expert without rows
 // exits before touching its weights.  SWIGLU gives a warp the gate row j and
-// the up row N/2 + j and writes silu(g) * u.
+// the up row N/2 + j and writes silu(g) * u.  For K <= 512 (at most 16 chunks
+// per row) each half-warp takes its own rows, so no lane idles.
 #include "common.cuh"
 #include "internal.h"
 
@@ -100,14 +101,20 @@ NVFP4_DEV void chunk_dot(const uint4& wq, const uint32_t (&xw)[16], float& p0, f
     }
 }
 
-template <int MT, int R, int QS, int J, int LAYOUT, typename OutT, int EPI>
+// HALF: each half-warp takes its own R rows (for K of at most 512, where a
+// row has no more 32-element chunks than 16 lanes can cover).
+template <int MT, int R, int QS, int J, int LAYOUT, typename OutT, int EPI, int HALF = 0>
 __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
     constexpr int RG = 8 / QS;                                    // row groups per CTA
-    constexpr int RW = (EPI == NVFP4_EPI_SWIGLU) ? 1 : R;         // output columns per warp
+    constexpr int RW = (EPI == NVFP4_EPI_SWIGLU) ? 1 : R;         // output columns per warp (half-warp)
+    constexpr int LW = HALF ? 16 : 32;                            // lanes per row group
     static_assert(EPI != NVFP4_EPI_SWIGLU || R == 2, "SwiGLU pairs one gate and one up row");
+    static_assert(!HALF || (QS == 1 && EPI == NVFP4_EPI_NONE), "half-warp rows: no K split, plain epilogue");
     __shared__ float red[8][R][MT];
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5, lane32 = threadIdx.x & 31;
+    const int lane = HALF ? (lane32 & 15) : lane32;               // lane within the row group
+    const int half = HALF ? (lane32 >> 4) : 0;
     const int g = warp / QS, q = warp % QS;
     const int64_t K = a.K;
     const int64_t nch = K >> 5;                                   // 32-element chunks per row
@@ -115,7 +122,7 @@ __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
     const int64_t ncols_out = (EPI == NVFP4_EPI_SWIGLU) ? a.N / 2 : a.N;
     const int64_t c_begin = nch * q / QS, c_end = nch * (q + 1) / QS;
 
-    const int64_t col0 = ((int64_t)blockIdx.y * RG + g) * RW;
+    const int64_t col0 = (((int64_t)blockIdx.y * RG + g) * (HALF ? 2 : 1) + half) * RW;
     const bool warp_active = col0 < ncols_out;
 
     int64_t row_begin, row_end;
@@ -161,13 +168,13 @@ __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
             for (int t = 0; t < MT; ++t) acc[i][t] = 0.0f;
 
         if (warp_active) {
-            for (int64_t cb = c_begin; cb < c_end; cb += 32 * J) {
+            for (int64_t cb = c_begin; cb < c_end; cb += LW * J) {
                 // issue every load of the batch first
                 uint4 wq[R][J];
                 uint16_t s2[R][J];
 #pragma unroll
                 for (int j = 0; j < J; ++j) {
-                    const int64_t c = cb + lane + 32 * j;
+                    const int64_t c = cb + lane + LW * j;
                     const bool ok = c < c_end;
 #pragma unroll
                     for (int i = 0; i < R; ++i) {
@@ -183,7 +190,7 @@ __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
                 }
 #pragma unroll
                 for (int j = 0; j < J; ++j) {
-                    const int64_t c = cb + lane + 32 * j;
+                    const int64_t c = cb + lane + LW * j;
                     if (c >= c_end) break;
 #pragma unroll
                     for (int t = 0; t < MT; ++t) {
@@ -208,7 +215,14 @@ __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
 #pragma unroll
         for (int i = 0; i < R; ++i)
 #pragma unroll
-            for (int t = 0; t < MT; ++t) acc[i][t] = warp_sum(acc[i][t]);
+            for (int t = 0; t < MT; ++t) {
+                if constexpr (HALF) {
+#pragma unroll
+                    for (int o = 8; o > 0; o >>= 1) acc[i][t] += __shfl_xor_sync(0xffffffffu, acc[i][t], o);
+                } else {
+                    acc[i][t] = warp_sum(acc[i][t]);
+                }
+            }
 
         if constexpr (QS > 1) {
             if (lane == 0) {
@@ -238,7 +252,7 @@ __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
             for (int i = 0; i < RW; ++i) {
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
-                    if (lane == ((i * MT + t) & 31) && t < nt && cvalid[i]) {
+                    if (lane == ((i * MT + t) & (LW - 1)) && t < nt && cvalid[i]) {
                         const float sc = gs * a.inv_scale[m0 + t];
                         float v;
                         if constexpr (EPI == NVFP4_EPI_SWIGLU) {
@@ -289,16 +303,17 @@ __global__ void __launch_bounds__(256) gemv_w4a16_odd_kernel(const GemvArgs a) {
     if (lane == 0) store_out<OutT>(reinterpret_cast<OutT*>(a.y) + m * a.ldy + n, acc * a.gs[0] * a.inv_scale[m]);
 }
 
-template <int MT, int R, int QS, int J, int LAYOUT, typename OutT, int EPI>
+template <int MT, int R, int QS, int J, int LAYOUT, typename OutT, int EPI, int HALF = 0>
 static int launch_cfg(const GemvArgs& a, cudaStream_t st) {
     constexpr int RG = 8 / QS;
     constexpr int RW = (EPI == NVFP4_EPI_SWIGLU) ? 1 : R;
+    constexpr int CPB = RG * RW * (HALF ? 2 : 1);  // output columns per CTA
     const int64_t ncols = (EPI == NVFP4_EPI_SWIGLU) ? a.N / 2 : a.N;
-    const int64_t tiles = (ncols + RG * RW - 1) / (RG * RW);
+    const int64_t tiles = (ncols + CPB - 1) / CPB;
     const int64_t gx = a.offsets ? (a.experts ? a.n_slots : a.E) : (a.M + MT - 1) / MT;
     if (tiles > 65535 || gx > 0x7fffffff) return NVFP4_ERR_SHAPE;
     dim3 grid((unsigned)gx, (unsigned)tiles);
-    gemv_w4a16_kernel<MT, R, QS, J, LAYOUT, OutT, EPI><<<grid, 256, 0, st>>>(a);
+    gemv_w4a16_kernel<MT, R, QS, J, LAYOUT, OutT, EPI, HALF><<<grid, 256, 0, st>>>(a);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 
@@ -316,6 +331,9 @@ static int launch_qs(const GemvArgs& a, cudaStream_t st) {
         // grouped (decode-time experts, a few rows each): two chunks in flight per
         // lane keep the register count, and so the resident warps per SM, up
         qs = nch >= 128 ? 2 : 1;
+        // short rows (K <= 512): each half-warp takes four rows of its own
+        if constexpr (EPI == NVFP4_EPI_NONE)
+            if (nch <= 16) return launch_cfg<MT, 4, 1, 1, LAYOUT, OutT, EPI, 1>(a, st);
         if (qs == 1) return launch_cfg<MT, 2, 1, 2, LAYOUT, OutT, EPI>(a, st);
         return launch_cfg<MT, 2, 2, 2, LAYOUT, OutT, EPI>(a, st);
     }
