@@ -23,8 +23,8 @@
 // Grouped form (mixture of experts; CHImp Alpha v1.0 model card, "How it fits
 // on one GPU": only the chosen experts are read): grid.x walks the experts,
 // expert e's rows are [offsets[e], offsets[e+1]); an expert without rows
-// exits before touching its weights.  SWIGLU gives a warp the gate row j and
-// the up row N/2 + j and writes silu(g) * u.  For K <= 512 (at most 16 chunks
+// exits before touching its weights.  SWIGLU gives a warp gate rows j and the
+// matching up rows N/2 + j and writes silu(g) * u.  For K <= 512 (at most 16 chunks
 // per row) each half-warp takes its own rows, so no lane idles.
 #include "common.cuh"
 #include "internal.h"
@@ -106,9 +106,9 @@ NVFP4_DEV void chunk_dot(const uint4& wq, const uint32_t (&xw)[16], float& p0, f
 template <int MT, int R, int QS, int J, int LAYOUT, typename OutT, int EPI, int HALF = 0>
 __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
     constexpr int RG = 8 / QS;                                    // row groups per CTA
-    constexpr int RW = (EPI == NVFP4_EPI_SWIGLU) ? 1 : R;         // output columns per warp (half-warp)
+    constexpr int RW = (EPI == NVFP4_EPI_SWIGLU) ? R / 2 : R;     // output columns per warp (half-warp)
     constexpr int LW = HALF ? 16 : 32;                            // lanes per row group
-    static_assert(EPI != NVFP4_EPI_SWIGLU || R == 2, "SwiGLU pairs one gate and one up row");
+    static_assert(EPI != NVFP4_EPI_SWIGLU || R % 2 == 0, "SwiGLU pairs gate rows with up rows");
     static_assert(!HALF || (QS == 1 && EPI == NVFP4_EPI_NONE), "half-warp rows: no K split, plain epilogue");
     __shared__ float red[8][R][MT];
 
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
         cvalid[i] = c < ncols_out;
         const int64_t cc = cvalid[i] ? c : (warp_active ? col0 : 0);
         wrow[i] = cc;
-        if constexpr (EPI == NVFP4_EPI_SWIGLU) wrow[1] = a.N / 2 + cc;
+        if constexpr (EPI == NVFP4_EPI_SWIGLU) wrow[RW + i] = a.N / 2 + cc;
     }
 
     const __half* xh = reinterpret_cast<const __half*>(a.xh);
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(256) gemv_w4a16_kernel(const GemvArgs a) {
                         const float sc = gs * a.inv_scale[m0 + t];
                         float v;
                         if constexpr (EPI == NVFP4_EPI_SWIGLU) {
-                            const float gg = acc[0][t] * sc, u = acc[1][t] * sc;
+                            const float gg = acc[i][t] * sc, u = acc[RW + i][t] * sc;
                             v = gg / (1.0f + expf(-gg)) * u;
                         } else {
                             v = acc[i][t] * sc;
@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(256) gemv_w4a16_odd_kernel(const GemvArgs a) {
 template <int MT, int R, int QS, int J, int LAYOUT, typename OutT, int EPI, int HALF = 0>
 static int launch_cfg(const GemvArgs& a, cudaStream_t st) {
     constexpr int RG = 8 / QS;
-    constexpr int RW = (EPI == NVFP4_EPI_SWIGLU) ? 1 : R;
+    constexpr int RW = (EPI == NVFP4_EPI_SWIGLU) ? R / 2 : R;
     constexpr int CPB = RG * RW * (HALF ? 2 : 1);  // output columns per CTA
     const int64_t ncols = (EPI == NVFP4_EPI_SWIGLU) ? a.N / 2 : a.N;
     const int64_t tiles = (ncols + CPB - 1) / CPB;
@@ -334,6 +334,11 @@ static int launch_qs(const GemvArgs& a, cudaStream_t st) {
         // short rows (K <= 512): each half-warp takes four rows of its own
         if constexpr (EPI == NVFP4_EPI_NONE)
             if (nch <= 16) return launch_cfg<MT, 4, 1, 1, LAYOUT, OutT, EPI, 1>(a, st);
+        // SwiGLU: two gate and two up rows per warp share each activation chunk
+        if constexpr (EPI == NVFP4_EPI_SWIGLU) {
+            if (qs == 1) return launch_cfg<MT, 4, 1, 2, LAYOUT, OutT, EPI>(a, st);
+            return launch_cfg<MT, 4, 2, 2, LAYOUT, OutT, EPI>(a, st);
+        }
         if (qs == 1) return launch_cfg<MT, 2, 1, 2, LAYOUT, OutT, EPI>(a, st);
         return launch_cfg<MT, 2, 2, 2, LAYOUT, OutT, EPI>(a, st);
     }
