@@ -11,8 +11,9 @@ linear.  Weights are quantized on the device by ``nvfp4_quantize`` and rotated
 over two copies (389 MB > the 126 MB L2), so every step streams from HBM.
 
 Also reported in the same JSON line (measured outside the headline's timed
-region): the decode sweep M in {1, 2, 4, 8, 16, 32} per shape, and whatever
-other sections the library supports (prefill W4A4 TFLOP/s, MoE).
+region): the decode sweep M in {1, 2, 4, 8, 16, 32} per shape, prefill W4A4
+TFLOP/s, the activation quantizer, one MoE layer, and the 64-layer decode stack
+(the four linears per layer chained through the library's rms / silu kernels).
 
 ``--impl reference`` times the CPU oracle (the method's plain restatement) on
 the same workload and metric, on this host's cores.  With more than one GPU
@@ -295,6 +296,10 @@ def run_native(args, rank, world, dist):
         extra["prefill"] = prefill_section(nv, torch, dev, layers)
         extra["quantize"] = quantize_section(nv, torch, dev)
         extra["moe_layer"] = moe_section(nv, torch, dev)
+        try:
+            extra["decode_stack"] = stack_section(nv, torch, dev, peak)
+        except Exception as exc:  # reported in the line; the headline above stands
+            extra["decode_stack"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -508,6 +513,93 @@ def moe_section(nv, torch, dev, reps=30):
                                 "GB/s": round(nbytes / (t * 1e-3) / 1e9, 1),
                                 "TFLOPs": round(flop / (t * 1e-3) / 1e12, 2)}
     del gu, dn
+    return out
+
+
+def stack_section(nv, torch, dev, peak_gbs, reps=10):
+    """The dense decode stack: 64 layers of the four 27B-shaped linears (12.46
+    GB of NVFP4 weights resident), each layer chained through the library's
+    glue kernels with attention left out:
+        q = QKV(x); o = O(rms(q[:, :5120])); g = GU(rms(o));
+        h = silu(g[:, :17408]) * g[:, 17408:]; x' = rms(Down(h))
+    One step is the whole stack for M tokens, captured once as a CUDA graph and
+    replayed; GB/s = (weight bytes + activation bytes read by the linears) /
+    step time.  Weights 0.02 N(0, 1) drawn on the device (seed 1000 + 4 i + j)
+    and quantized there; x0 N(0, 1) renormalised."""
+    L = 64
+    layers = []
+    for i in range(L):
+        mats = {}
+        for j, (name, K, N, _) in enumerate(SHAPES):
+            gen = torch.Generator(device=dev)
+            gen.manual_seed(1000 + 4 * i + j)
+            w = 0.02 * torch.randn((N, K), generator=gen, device=dev)
+            mats[name] = nv.nvfp4_quantize(w, sf_layout=nv.SF_TILED)
+            del w
+        layers.append(mats)
+    torch.cuda.synchronize()
+    kq, nq = SHAPES[0][1], SHAPES[0][2]
+    ng = SHAPES[2][2]
+    out = {"layers": L, "weight_bytes": L * sum(N * K // 2 + N * K // 16 for _, K, N, _ in SHAPES),
+           "timing": "CUDA-graph replay of the 64-layer step, events on the launching stream", "runs": {}}
+    stream = torch.cuda.current_stream()
+    side = torch.cuda.Stream(device=dev)
+    for M in (1, 8, 32):
+        gx = torch.Generator(device=dev)
+        gx.manual_seed(999)
+        x = nv.nvfp4_rms_norm(torch.randn((M, kq), generator=gx, device=dev))
+        bufs = {name: torch.empty((M, N), dtype=torch.float32, device=dev) for name, _, N, _ in SHAPES}
+        ws = {name: torch.empty(max(16, int(nv.lib().nvfp4_linear_workspace(M, K, N, nv.MODE_W4A16))),
+                                dtype=torch.uint8, device=dev) for name, K, N, _ in SHAPES}
+        o_in = torch.empty((M, kq), dtype=torch.bfloat16, device=dev)
+        gu_in = torch.empty((M, kq), dtype=torch.bfloat16, device=dev)
+        h = torch.empty((M, ng // 2), dtype=torch.bfloat16, device=dev)
+        x_next = torch.empty((M, kq), dtype=torch.bfloat16, device=dev)
+
+        def lin(xin, li, name):
+            c, s, g = layers[li][name]
+            return nv.nvfp4_linear(xin, c, s, g, w_sf_layout=nv.SF_TILED, y=bufs[name], mode=nv.MODE_W4A16,
+                                   ws=ws[name])
+
+        def step():
+            cur = x
+            for li in range(L):
+                q = lin(cur, li, "qkv")
+                nv.nvfp4_rms_norm(q, cols=kq, y=o_in)
+                o = lin(o_in, li, "o_proj")
+                nv.nvfp4_rms_norm(o, y=gu_in)
+                g = lin(gu_in, li, "gate_up")
+                nv.nvfp4_silu_mul(g, h=h)
+                d = lin(h, li, "down")
+                nv.nvfp4_rms_norm(d, y=x_next)
+                cur = x_next
+
+        step()
+        torch.cuda.synchronize()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=side):
+                step()
+        stream.wait_stream(side)
+        for _ in range(3):
+            gr.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            gr.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        nbytes = L * sum(decode_bytes(M, K, N) for _, K, N, _ in SHAPES)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        x_out = x_next.float()
+        out["runs"][f"M{M}"] = {"ms_per_step": round(ms, 4), "us_per_layer": round(ms * 1e3 / L, 2),
+                                "GB/s": round(gbs, 1), "frac_of_peak": round(gbs / peak_gbs, 4),
+                                "final_rms": round(float(x_out.pow(2).mean().sqrt()), 4),
+                                "finite": bool(torch.isfinite(x_out).all())}
+        del gr
     return out
 
 

@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
             "nvfp4_linear_workspace": (sz, [i64, i64, i64, i]),
             "nvfp4_linear": (i, [p, i, i64, i64, p, p, i, p, i64, p, i, i, p, sz, p]),
             "nvfp4_linear_w4a4q": (i, [p, p, p, i64, i64, p, p, p, i64, p, i, p]),
+            "nvfp4_rms_norm": (i, [p, i, i64, i64, i64, p, p]),
+            "nvfp4_silu_mul": (i, [p, i, i64, i64, p, p]),
             "moe_route_topk_workspace": (sz, [i64, i32, i32]),
             "moe_route_topk": (i, [p, p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p, sz, p]),
             "moe_route_topk_noalloc": (i, [p, p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p]),
@@ -123,6 +125,31 @@ def nvfp4_quantize(x: torch.Tensor, gs_in: torch.Tensor | None = None, sf_layout
     _check(lib().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, _ptr(gs_in), sf_layout, _ptr(codes),
                                 _ptr(scales), _ptr(gs_out), _ptr(ws), wsb, _stream()), "nvfp4_quantize")
     return codes, scales, gs_out
+
+
+def nvfp4_rms_norm(x: torch.Tensor, cols: int | None = None, y=None):
+    """``bf16(v / sqrt(mean(v^2)))`` for the first ``cols`` columns of each row v of
+    ``x [rows, ld]`` (fp32 or bf16, rows contiguous); returns ``y [rows, cols]`` bf16."""
+    rows, ld = x.shape
+    if x.stride(1) != 1 or x.stride(0) != ld:
+        raise ValueError("x must be a contiguous [rows, ld] tensor")
+    cols = ld if cols is None else int(cols)
+    if y is None:
+        y = torch.empty((rows, cols), dtype=torch.bfloat16, device=x.device)
+    _check(lib().nvfp4_rms_norm(_ptr(x), _dtype_code(x), rows, cols, ld, _ptr(y), _stream()), "nvfp4_rms_norm")
+    return y
+
+
+def nvfp4_silu_mul(g: torch.Tensor, h=None):
+    """``bf16(silu(g[:, :n]) * g[:, n:])`` for ``g [rows, 2n]`` (fp32 or bf16, contiguous)."""
+    rows, w = g.shape
+    if not g.is_contiguous() or w % 2:
+        raise ValueError("g must be a contiguous [rows, 2n] tensor")
+    half = w // 2
+    if h is None:
+        h = torch.empty((rows, half), dtype=torch.bfloat16, device=g.device)
+    _check(lib().nvfp4_silu_mul(_ptr(g), _dtype_code(g), rows, half, _ptr(h), _stream()), "nvfp4_silu_mul")
+    return h
 
 
 def nvfp4_linear(x: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, w_gs: torch.Tensor,

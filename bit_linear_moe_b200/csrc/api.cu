@@ -274,6 +274,34 @@ int nvfp4_linear_w4a4q(const uint8_t* x_codes, const uint8_t* x_scales, const fl
                             device_status_ptr(), (cudaStream_t)stream);
 }
 
+// ---- decode-stack glue ---------------------------------------------------------------
+
+static bool float_dtype_ok(int d) { return d == NVFP4_DTYPE_F32 || d == NVFP4_DTYPE_BF16; }
+static bool elem_aligned(const void* p, int d) {
+    return ((uintptr_t)p & (uintptr_t)(d == NVFP4_DTYPE_F32 ? 3 : 1)) == 0;
+}
+
+int nvfp4_rms_norm(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld, void* y, void* stream) {
+    if (!x || !y) return NVFP4_ERR_NULL;
+    if (!float_dtype_ok(x_dtype)) return NVFP4_ERR_DTYPE;
+    if (rows < 1 || cols < 1 || ld < cols || rows > ((int64_t)1 << 31) - 1 || cols > ((int64_t)1 << 31) ||
+        ld > ((int64_t)1 << 40) / rows)
+        return NVFP4_ERR_SHAPE;
+    if (!elem_aligned(x, x_dtype) || !elem_aligned(y, NVFP4_DTYPE_BF16)) return NVFP4_ERR_ALIGN;
+    NVFP4_TRY(check_arch());
+    return launch_rms_norm(x, x_dtype, rows, cols, ld, y, (cudaStream_t)stream);
+}
+
+int nvfp4_silu_mul(const void* g, int g_dtype, int64_t rows, int64_t half, void* h, void* stream) {
+    if (!g || !h) return NVFP4_ERR_NULL;
+    if (!float_dtype_ok(g_dtype)) return NVFP4_ERR_DTYPE;
+    if (rows < 1 || half < 1 || rows > ((int64_t)1 << 31) || half > ((int64_t)1 << 40) / rows)
+        return NVFP4_ERR_SHAPE;
+    if (!elem_aligned(g, g_dtype) || !elem_aligned(h, NVFP4_DTYPE_BF16)) return NVFP4_ERR_ALIGN;
+    NVFP4_TRY(check_arch());
+    return launch_silu_mul(g, g_dtype, rows, half, h, (cudaStream_t)stream);
+}
+
 // ---- MoE routing -------------------------------------------------------------------
 
 static int64_t perm_blocks(int64_t T) { return (T + kPermBlockTokens - 1) / kPermBlockTokens; }

@@ -16,6 +16,10 @@ inline void set_pdl_attr(cudaLaunchAttribute& a) {
     a.val.programmaticStreamSerializationAllowed = 1;
 }
 
+// stack.cu: decode-stack glue (bf16 outputs)
+int launch_rms_norm(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld, void* y, cudaStream_t st);
+int launch_silu_mul(const void* g, int g_dtype, int64_t rows, int64_t half, void* h, cudaStream_t st);
+
 // quantize.cu
 int launch_amax(const void* x, int x_dtype, int64_t n, unsigned* amax_bits, cudaStream_t st);
 // src_rows (nullable): dst row r quantizes source row src_rows[r]; -1 = zero row.

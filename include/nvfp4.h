@@ -171,6 +171,25 @@ int nvfp4_linear_w4a4q(const uint8_t* x_codes, const uint8_t* x_scales, const fl
                        const uint8_t* w_codes, const uint8_t* w_scales, const float* w_gs, int64_t N,
                        void* y, int y_dtype, void* stream);
 
+/* ---- nvfp4_rms_norm / nvfp4_silu_mul -------------------------------------
+ * The glue between the linears of a dense decode stack (Ignis README, "The
+ * decode round": a decode step streams the whole stack's weights once).  The
+ * pages leave the chaining open; with attention left out each layer is
+ *     q = QKV(x); o = O(rms(q[:, :K_o])); g = GU(rms(o));
+ *     h = silu(g[:, :N/2]) * g[:, N/2:]; x' = rms(Down(h))
+ * nvfp4_rms_norm:  y[r, c] = bf16(x[r, c] / sqrt(mean_c x[r, c]^2)), rounded
+ *   to nearest even; an all-zero row gives zeros.
+ *   x      rows of `cols` elements, row r starting at element r * ld
+ *          (ld >= cols, so a column slice of a wider matrix is read in place);
+ *          x_dtype F32 or BF16
+ *   y      [rows, cols] bf16, densely packed
+ * nvfp4_silu_mul:  h[r, j] = bf16(silu(g[r, j]) * g[r, half + j]),
+ *   silu(v) = v / (1 + e^-v)
+ *   g      [rows, 2 * half], g_dtype F32 or BF16;  h  [rows, half] bf16
+ * Element-size alignment only; no workspace. */
+int nvfp4_rms_norm(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld, void* y, void* stream);
+int nvfp4_silu_mul(const void* g, int g_dtype, int64_t rows, int64_t half, void* h, void* stream);
+
 /* ---- moe_route_topk ------------------------------------------------------
  * Router of a routed mixture-of-experts layer (CHImp Alpha v1.0 model card,
  * "How it fits on one GPU": 10 of 512 experts per token).

@@ -150,3 +150,34 @@ def test_grouped_validation(L):
     assert g(K=48) == nv.ERR_SHAPE
     if not torch.cuda.is_available():
         assert g() == nv.ERR_ARCH
+
+
+def test_stack_glue_validation(L):
+    ODD = ctypes.c_void_p(0x10001)
+
+    def rms(**kw):
+        a = dict(x=FAKE, xd=nv.DTYPE_F32, rows=2, cols=64, ld=128, y=FAKE2)
+        a.update(kw)
+        return L.nvfp4_rms_norm(a["x"], a["xd"], a["rows"], a["cols"], a["ld"], a["y"], None)
+
+    assert rms(x=None) == nv.ERR_NULL
+    assert rms(y=None) == nv.ERR_NULL
+    assert rms(xd=3) == nv.ERR_DTYPE
+    assert rms(rows=0) == nv.ERR_SHAPE
+    assert rms(cols=0) == nv.ERR_SHAPE
+    assert rms(ld=63) == nv.ERR_SHAPE
+    assert rms(x=ctypes.c_void_p(0x10002)) == nv.ERR_ALIGN       # fp32 rows need 4-byte alignment
+    assert rms(x=ctypes.c_void_p(0x10002), xd=nv.DTYPE_BF16) != nv.ERR_ALIGN
+    assert rms(y=ODD) == nv.ERR_ALIGN
+
+    def silu(**kw):
+        a = dict(g=FAKE, gd=nv.DTYPE_BF16, rows=2, half=64, h=FAKE2)
+        a.update(kw)
+        return L.nvfp4_silu_mul(a["g"], a["gd"], a["rows"], a["half"], a["h"], None)
+
+    assert silu(g=None) == nv.ERR_NULL
+    assert silu(gd=7) == nv.ERR_DTYPE
+    assert silu(half=0) == nv.ERR_SHAPE
+    assert silu(g=ODD) == nv.ERR_ALIGN
+    if not torch.cuda.is_available():
+        assert rms() == nv.ERR_ARCH and silu() == nv.ERR_ARCH

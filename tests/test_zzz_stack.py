@@ -1,0 +1,105 @@
+"""GPU decode-stack glue (rms renormalisation, silu * up) against the oracle,
+and one stack layer on small shapes checked stage by stage (each stage on the
+GPU's own input to it).  bf16 outputs may differ from the oracle's bf16 by one
+bf16 step: the GPU sums in fp32, in another order, before the same rounding."""
+import numpy as np
+import pytest
+import torch
+
+import bit_linear_moe_b200 as nv
+import oracle
+from oracle import stack as ost
+from bit_linear_moe_b200 import synth
+from nvfp4_checks import assert_within_bound, bf16_ulp, rowmajor_to_tiled
+
+pytestmark = pytest.mark.gpu
+
+
+def _close_bf16(got, ref, what):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.abs(got - ref)
+    lim = bf16_ulp(ref) + 1e-30
+    assert (err <= lim).all(), f"{what}: {(err > lim).sum()} elements off by more than one bf16 step"
+
+
+@pytest.mark.parametrize("rows,cols,ld,dtype", [(1, 5120, 10240, torch.float32), (8, 5120, 5120, torch.bfloat16),
+                                                (3, 100, 100, torch.float32), (32, 5120, 5120, torch.float32),
+                                                (4, 777, 800, torch.bfloat16)])
+def test_rms_norm(rows, cols, ld, dtype):
+    rng = np.random.default_rng(rows * 7 + cols)
+    x = (rng.standard_normal((rows, ld)) * rng.uniform(0.01, 100, (rows, 1))).astype(np.float32)
+    if rows > 2:
+        x[1] = 0.0                                  # an all-zero row stays zero
+    xd = torch.from_numpy(x).to(dtype).cuda()
+    y = nv.nvfp4_rms_norm(xd, cols=cols)
+    torch.cuda.synchronize()
+    xin = xd.float().cpu().numpy()[:, :cols]
+    ref = ost.rms_norm(xin)
+    _close_bf16(y.float().cpu().numpy(), ref, f"rms {rows}x{cols}")
+    if rows > 2:
+        assert not y[1].float().any()
+
+
+@pytest.mark.parametrize("rows,half,dtype", [(1, 17408, torch.float32), (32, 17408, torch.bfloat16),
+                                             (5, 33, torch.float32)])
+def test_silu_mul(rows, half, dtype):
+    rng = np.random.default_rng(rows + half)
+    g = (4 * rng.standard_normal((rows, 2 * half))).astype(np.float32)
+    gd = torch.from_numpy(g).to(dtype).cuda()
+    h = nv.nvfp4_silu_mul(gd)
+    torch.cuda.synchronize()
+    ref = ost.silu_mul(gd.float().cpu().numpy())
+    _close_bf16(h.float().cpu().numpy(), ref, f"silu_mul {rows}x{half}")
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_stack_layer_small(M):
+    """One layer of the stack on small shapes: hidden 512, QKV 1024, GU 2 x 768."""
+    d, nq, ni = 512, 1024, 768
+    rng = np.random.default_rng(900 + M)
+    shapes = {"qkv": (nq, d), "o": (d, d), "gu": (2 * ni, d), "down": (d, ni)}
+    q_w = {k: oracle.quantize(synth.weight(np.random.default_rng([900, i]), n, kk))
+           for i, (k, (n, kk)) in enumerate(shapes.items())}
+    dev_w = {}
+    for k, (c, s, g) in q_w.items():
+        n, kk = shapes[k]
+        dev_w[k] = (torch.from_numpy(np.ascontiguousarray(c)).cuda(),
+                    torch.from_numpy(np.ascontiguousarray(rowmajor_to_tiled(s, n, kk)).ravel()).cuda(),
+                    torch.tensor([g], dtype=torch.float32, device="cuda"))
+
+    def lin(x_bf16, k):
+        c, s, g = dev_w[k]
+        return nv.nvfp4_linear(x_bf16, c, s, g, w_sf_layout=nv.SF_TILED, y_dtype=torch.float32,
+                               mode=nv.MODE_W4A16)
+
+    x0 = ost.rms_norm(rng.standard_normal((M, d)).astype(np.float32))
+    x = torch.from_numpy(x0).to(torch.bfloat16).cuda()
+    q = lin(x, "qkv")
+    o_in = nv.nvfp4_rms_norm(q, cols=d)
+    o = lin(o_in, "o")
+    gu_in = nv.nvfp4_rms_norm(o)
+    g = lin(gu_in, "gu")
+    h = nv.nvfp4_silu_mul(g)
+    dn = lin(h, "down")
+    x1 = nv.nvfp4_rms_norm(dn)
+    torch.cuda.synchronize()
+
+    def host(t):
+        return t.float().cpu().numpy()
+
+    ref, ad = oracle.linear_w4a16(x0, *q_w["qkv"])
+    assert_within_bound(q, ref, ad, False, "qkv")
+    _close_bf16(host(o_in), ost.rms_norm(host(q)[:, :d]), "rms(q slice)")
+    ref, ad = oracle.linear_w4a16(host(o_in), *q_w["o"])
+    assert_within_bound(o, ref, ad, False, "o")
+    _close_bf16(host(gu_in), ost.rms_norm(host(o)), "rms(o)")
+    ref, ad = oracle.linear_w4a16(host(gu_in), *q_w["gu"])
+    assert_within_bound(g, ref, ad, False, "gate/up")
+    _close_bf16(host(h), ost.silu_mul(host(g)), "silu * up")
+    ref, ad = oracle.linear_w4a16(host(h), *q_w["down"])
+    assert_within_bound(dn, ref, ad, False, "down")
+    _close_bf16(host(x1), ost.rms_norm(host(dn)), "rms(down)")
+    # the renormalised output has mean square 1 up to the bf16 rounding
+    ms = np.mean(host(x1).astype(np.float64) ** 2, axis=1)
+    assert np.allclose(ms, 1.0, atol=2e-2)
