@@ -181,3 +181,18 @@ def test_stack_glue_validation(L):
     assert silu(g=ODD) == nv.ERR_ALIGN
     if not torch.cuda.is_available():
         assert rms() == nv.ERR_ARCH and silu() == nv.ERR_ARCH
+
+
+def test_noalloc_scratch_limit(L):
+    """The allocation-free router needs ceil(T/32) * E * 8 bytes of its 1 MiB
+    scratch (plus T * E * 4 without a logits buffer) and says so before
+    touching the device."""
+    def route(T, logits):
+        return L.moe_route_topk_noalloc(FAKE, FAKE2, None, T, 2048, 512, 10, logits, FAKE, FAKE, FAKE, FAKE,
+                                        FAKE, FAKE, None)
+
+    assert route(8192 + 1, FAKE) == nv.ERR_WORKSPACE            # 257 blocks x 512 x 8 > 1 MiB
+    assert route(513, None) == nv.ERR_WORKSPACE                 # 513 x 512 x 4 B of logits alone > 1 MiB
+    if not torch.cuda.is_available():
+        assert route(8192, FAKE) == nv.ERR_ARCH                 # fits: validation passes, then no B200
+        assert route(32, None) == nv.ERR_ARCH
