@@ -625,6 +625,90 @@ def quantize_section(nv, torch, dev, reps=30):
     return out
 
 
+# ------------------------------------------------------------ profile cases ----
+
+CASES = ("decode_m1", "skinny_m4", "prefill_m2048", "quantize_m2048", "moe_t1", "moe_t32", "moe_t4096",
+         "stack_glue_m1")
+
+
+def profile_case(args):
+    """One small workload, launched eagerly ``--steps`` times, for a profiler to
+    capture a few launches of one kernel (a few GB on the device at most)."""
+    import torch
+    import bit_linear_moe_b200 as nv
+    from bit_linear_moe_b200 import synth
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    case = args.case
+    shapes = {name: (K, N) for name, K, N, _ in SHAPES}
+
+    def qw(K, N):
+        return nv.nvfp4_quantize(0.02 * torch.randn((N, K), generator=gen, device=dev), sf_layout=nv.SF_TILED)
+
+    if case in ("decode_m1", "skinny_m4", "stack_glue_m1"):
+        M = 4 if case == "skinny_m4" else 1
+        ws_ = {name: qw(K, N) for name, (K, N) in shapes.items()}
+        xs = {name: torch.randn((M, K), generator=gen, device=dev).to(torch.bfloat16) for name, (K, N) in shapes.items()}
+
+        def run():
+            for name, (K, N) in shapes.items():
+                c, s_, g = ws_[name]
+                y = nv.nvfp4_linear(xs[name], c, s_, g, w_sf_layout=nv.SF_TILED, mode=nv.MODE_W4A16)
+                if case == "stack_glue_m1":
+                    if name == "gate_up":
+                        nv.nvfp4_silu_mul(y)
+                    else:
+                        nv.nvfp4_rms_norm(y, cols=min(y.shape[1], 5120))
+    elif case == "prefill_m2048":
+        K, N = shapes["qkv"]
+        c, s_, g = qw(K, N)
+        x = torch.randn((2048, K), generator=gen, device=dev).to(torch.bfloat16)
+        xc, xs_, xg = nv.nvfp4_quantize(x, sf_layout=nv.SF_TILED)
+
+        def run():
+            nv.nvfp4_linear_w4a4q(xc, xs_, xg, c, s_, g)
+    elif case == "quantize_m2048":
+        x = torch.randn((2048, 5120), generator=gen, device=dev).to(torch.bfloat16)
+
+        def run():
+            nv.nvfp4_quantize(x, sf_layout=nv.SF_TILED)
+    else:
+        E, H, I, k = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_K
+        T = int(case[len("moe_t"):])
+        mode = nv.MODE_W4A4 if T > 32 else nv.MODE_W4A16
+
+        def stack(n, kk):
+            sb = nv.nvfp4_scales_bytes(n, kk, nv.SF_TILED)
+            codes = torch.empty((E, n, kk // 2), dtype=torch.uint8, device=dev)
+            scales = torch.empty(E * sb, dtype=torch.uint8, device=dev)
+            gs = torch.empty(E, dtype=torch.float32, device=dev)
+            for e in range(E):
+                nv.nvfp4_quantize(0.02 * torch.randn((n, kk), generator=gen, device=dev), sf_layout=nv.SF_TILED,
+                                  codes=codes[e], scales=scales[e * sb:(e + 1) * sb], gs_out=gs[e:e + 1])
+            return codes, scales, gs
+
+        gu, dn = stack(2 * I, H), stack(H, I)
+        wr = (0.02 * torch.randn((E, H), generator=gen, device=dev)).to(torch.bfloat16)
+        h = torch.randn((T, H), generator=gen, device=dev).to(torch.bfloat16)
+        R = T * k
+
+        def run():
+            r = nv.moe_route_topk(h, wr, k)
+            a = nv.moe_grouped_linear(h, r["expert_offsets"], *gu, R, perm_tok=r["perm_tok"], gather=True,
+                                      w_sf_layout=nv.SF_TILED, epilogue=nv.EPI_SWIGLU, y_dtype=torch.bfloat16,
+                                      mode=mode)
+            nv.moe_grouped_linear(a, r["expert_offsets"], *dn, R, gather=False, w_sf_layout=nv.SF_TILED,
+                                  epilogue=nv.EPI_COMBINE, topk_w=r["topk_w"], row_of=r["row_of"], k=k,
+                                  mode=mode)
+    for _ in range(args.steps):
+        run()
+    torch.cuda.synchronize()
+    assert nv.nvfp4_read_device_status() == nv.OK
+    print(json.dumps({"case": case, "steps": args.steps, "ok": True}))
+
+
 # --------------------------------------------------------------- reference ----
 
 def oracle_decode_sample(min_seconds: float = 10.0, row_frac: int = 1):
@@ -694,7 +778,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--quick", action="store_true", help="headline only (no sweeps, no CPU baseline)")
+    ap.add_argument("--case", choices=CASES, default=None,
+                    help="run one small workload eagerly --steps times (for profiler captures) and exit")
     args = ap.parse_args()
+    if args.case:
+        profile_case(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
 

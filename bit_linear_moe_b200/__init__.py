@@ -51,6 +51,7 @@ def lib() -> ctypes.CDLL:
             "nvfp4_version": (i, []),
             "nvfp4_scales_bytes": (sz, [i64, i64, i]),
             "nvfp4_read_device_status": (i, [p, p]),
+            "nvfp4_debug_wait_timeout": (i, [i64, p]),
             "nvfp4_quantize_workspace": (sz, [i64, i64]),
             "nvfp4_quantize": (i, [p, i, i64, i64, p, i, p, p, p, p, sz, p]),
             "nvfp4_linear_workspace": (sz, [i64, i64, i64, i]),
@@ -62,6 +63,11 @@ def lib() -> ctypes.CDLL:
             "moe_route_topk": (i, [p, p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p, sz, p]),
             "moe_route_topk_noalloc": (i, [p, p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p]),
             "moe_grouped_linear_workspace": (sz, [i64, i64, i64, i32, i32, i, i]),
+            "nvfp4_linear_w4a4_ws_layout": (i, [i64, i64, p]),
+            "moe_layer_decode_workspace": (sz, [i64, i64, i64, i32, i32]),
+            "moe_layer_decode": (i, [p, p, p, i64, i64, i32, i32, p, p, p, i64, p, p, p, p, p, p, p, p, i, p, sz,
+                                     p]),
+            "moe_grouped_linear_w4a4_ws_layout": (i, [i64, i64, i64, i32, i32, i, p]),
             "moe_grouped_linear": (i, [p, i, i64, i, p, p, i32, i64, p, p, i, p, i64, i, p, p, i32, p, i, i,
                                        p, sz, p]),
         }
@@ -247,6 +253,57 @@ def moe_grouped_linear(x: torch.Tensor, expert_offsets: torch.Tensor, w_codes: t
                                     N, epilogue, _ptr(topk_w), _ptr(row_of), k, _ptr(y), _dtype_code(y), mode,
                                     _ptr(ws), wsb, _stream()), "moe_grouped_linear")
     return y
+
+
+def moe_layer_decode(h: torch.Tensor, w_router: torch.Tensor, k: int, gate_up, down, logit_bias=None,
+                     y=None, y_dtype=torch.float32, want_logits: bool = False, want_routing: bool = False,
+                     want_a: bool = False, ws=None):
+    """One expert layer for a decode batch (T <= 32): ``gate_up`` and ``down`` are
+    the stacked ``(codes, TILED scales, gs)`` of the experts.  Returns ``y``, or
+    ``(y, extras)`` with the requested ``logits``, ``topk_idx``/``topk_w`` and ``a``."""
+    T, H = h.shape
+    E = w_router.shape[0]
+    I = gate_up[0].shape[1] // 2
+    dev = h.device
+    if y is None:
+        y = torch.empty((T, H), dtype=y_dtype, device=dev)
+    ex = {}
+    if want_logits:
+        ex["logits"] = torch.empty((T, E), dtype=torch.float32, device=dev)
+    if want_routing:
+        ex["topk_idx"] = torch.empty((T, k), dtype=torch.int32, device=dev)
+        ex["topk_w"] = torch.empty((T, k), dtype=torch.float32, device=dev)
+    if want_a:
+        ex["a"] = torch.empty((T * k, I), dtype=torch.bfloat16, device=dev)
+    ws, wsb = _workspace(int(lib().moe_layer_decode_workspace(T, H, I, E, k)), dev, ws)
+    _check(lib().moe_layer_decode(_ptr(h), _ptr(w_router), _ptr(logit_bias), T, H, E, k, _ptr(gate_up[0]),
+                                  _ptr(gate_up[1]), _ptr(gate_up[2]), I, _ptr(down[0]), _ptr(down[1]),
+                                  _ptr(down[2]), _ptr(ex.get("logits")), _ptr(ex.get("topk_idx")),
+                                  _ptr(ex.get("topk_w")), _ptr(ex.get("a")), _ptr(y), _dtype_code(y), _ptr(ws),
+                                  wsb, _stream()), "moe_layer_decode")
+    return (y, ex) if ex else y
+
+
+def nvfp4_linear_w4a4_ws_layout(M: int, K: int) -> dict:
+    """Byte offsets, inside a W4A4 ``nvfp4_linear`` workspace, of the quantized
+    activations the call leaves there: ``gs_x``, ``codes``, ``scales``."""
+    out = (ctypes.c_int64 * 3)()
+    _check(lib().nvfp4_linear_w4a4_ws_layout(M, K, out), "nvfp4_linear_w4a4_ws_layout")
+    return dict(zip(("gs_x", "codes", "scales"), (int(v) for v in out)))
+
+
+def moe_grouped_linear_w4a4_ws_layout(R: int, K: int, N: int, E: int, k: int, epilogue: int) -> dict:
+    """Byte offsets, inside a W4A4 ``moe_grouped_linear`` workspace, of the padded
+    permuted activations the call leaves there (see include/nvfp4.h)."""
+    out = (ctypes.c_int64 * 6)()
+    _check(lib().moe_grouped_linear_w4a4_ws_layout(R, K, N, E, k, epilogue, out),
+           "moe_grouped_linear_w4a4_ws_layout")
+    return dict(zip(("gs_x", "pad_off", "src_rows", "codes", "scales", "rows_pad"), (int(v) for v in out)))
+
+
+def nvfp4_debug_wait_timeout(limit_cycles: int):
+    """Launch the library's wait-timeout probe (a bounded wait that runs out)."""
+    _check(lib().nvfp4_debug_wait_timeout(int(limit_cycles), _stream()), "nvfp4_debug_wait_timeout")
 
 
 def nvfp4_read_device_status() -> int:

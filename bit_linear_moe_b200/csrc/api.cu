@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdlib.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -13,42 +15,40 @@ __device__ int g_device_status = 0;
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
-// Device address of the status word, looked up once per device.
+// Device address of the status word, looked up once per device (the slots are
+// atomic: several host threads may make their first call at once; each stores
+// the same address).  A device reset invalidates the cached address.
 int* device_status_ptr() {
-    static int* cache[64] = {nullptr};
+    static std::atomic<int*> cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!cache[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
-        cache[dev] = (int*)p;
+    int* p = cache[dev].load(std::memory_order_acquire);
+    if (!p) {
+        void* q = nullptr;
+        if (cudaGetSymbolAddress(&q, g_device_status) != cudaSuccess) return nullptr;
+        p = (int*)q;
+        cache[dev].store(p, std::memory_order_release);
     }
-    return cache[dev];
+    return p;
 }
 static size_t align256(size_t n) { return (n + 255) & ~(size_t)255; }
 
-bool pdl_enabled() {
-    static const bool on = [] {
-        const char* e = getenv("NVFP4_PDL");
-        return !(e && e[0] == '0');
-    }();
-    return on;
-}
-
 // The current device must be sm_100 (B200 / GB200 class).  Cached per device.
 static int check_arch() {
-    static int cache[64] = {0};  // 0 unknown, 1 ok, 2 bad
+    static std::atomic<int> cache[64];  // 0 unknown, 1 ok, 2 bad
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NVFP4_ERR_ARCH;
     if (dev < 0 || dev >= 64) return NVFP4_ERR_ARCH;
-    if (cache[dev] == 0) {
+    int c = cache[dev].load(std::memory_order_relaxed);
+    if (c == 0) {
         int major = 0, minor = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
             return NVFP4_ERR_ARCH;
-        cache[dev] = (major == 10 && minor == 0) ? 1 : 2;
+        c = (major == 10 && minor == 0) ? 1 : 2;
+        cache[dev].store(c, std::memory_order_relaxed);
     }
-    return cache[dev] == 1 ? NVFP4_OK : NVFP4_ERR_ARCH;
+    return c == 1 ? NVFP4_OK : NVFP4_ERR_ARCH;
 }
 
 static bool dtype_ok(int d) { return d == NVFP4_DTYPE_F32 || d == NVFP4_DTYPE_BF16; }
@@ -82,9 +82,7 @@ struct GroupedW4A4Ws {
     int32_t* src_rows;
     uint8_t* codes;
     uint8_t* scales;
-    float* yacc;
-    int32_t* tok_of;
-    float* w_of;
+    __nv_bfloat16* d;  // COMBINE: the experts' rows [R, N] before the weighted sum
     size_t bytes;
 };
 static GroupedW4A4Ws grouped_w4a4_ws(void* base, int64_t R, int64_t K, int64_t N, int32_t E, int32_t k,
@@ -101,11 +99,7 @@ static GroupedW4A4Ws grouped_w4a4_ws(void* base, int64_t R, int64_t K, int64_t N
     w.src_rows = (int32_t*)take((size_t)rp * 4);
     w.codes = (uint8_t*)take((size_t)(rp * K / 2));
     w.scales = (uint8_t*)take(scales_bytes(rp, K, NVFP4_SF_TILED));
-    if (epilogue == NVFP4_EPI_COMBINE && k > 0) {
-        w.yacc = (float*)take((size_t)(R / k) * (size_t)N * 4);
-        w.tok_of = (int32_t*)take((size_t)R * 4);
-        w.w_of = (float*)take((size_t)R * 4);
-    }
+    if (epilogue == NVFP4_EPI_COMBINE) w.d = (__nv_bfloat16*)take((size_t)R * (size_t)N * 2);
     w.bytes = off;
     return w;
 }
@@ -259,6 +253,15 @@ int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t
     return launch_gemv_w4a16(a, st);
 }
 
+int nvfp4_linear_w4a4_ws_layout(int64_t M, int64_t K, int64_t* offsets) {
+    if (!offsets) return NVFP4_ERR_NULL;
+    if (M < 1 || K < 256 || K % 256 || M > ((int64_t)1 << 31) || K > ((int64_t)1 << 24)) return NVFP4_ERR_SHAPE;
+    offsets[0] = 16;                                          // gs_x
+    offsets[1] = 256;                                         // codes [M, K/2]
+    offsets[2] = 256 + (int64_t)align256((size_t)(M * K / 2));  // TILED scales
+    return NVFP4_OK;
+}
+
 int nvfp4_linear_w4a4q(const uint8_t* x_codes, const uint8_t* x_scales, const float* x_gs, int64_t M, int64_t K,
                        const uint8_t* w_codes, const uint8_t* w_scales, const float* w_gs, int64_t N, void* y,
                        int y_dtype, void* stream) {
@@ -338,6 +341,101 @@ int moe_route_topk(const void* h, const void* w_router, const float* logit_bias,
     return launch_perm_scatter(topk_idx, T, E, k, blk_base, perm_tok, perm_slot, row_of, st);
 }
 
+// ---- MoE layer for a decode batch --------------------------------------------------
+
+struct MoeDecodeWs {
+    float* logits;
+    int32_t* topk_idx;
+    float* topk_w;
+    int32_t* n_groups;
+    int32_t* groups;
+    int32_t* perm_t;
+    int32_t* perm_j;
+    int32_t* cnt;
+    void* a;
+    float* d;
+    size_t bytes;
+};
+static MoeDecodeWs moe_decode_ws(void* base, int64_t T, int64_t H, int64_t I, int32_t E, int32_t k) {
+    MoeDecodeWs w{};
+    char* p = (char*)base;
+    size_t off = 0;
+    auto take = [&](size_t n) { char* q = p ? p + off : nullptr; off += align256(n); return q; };
+    const size_t R = (size_t)(T * k);
+    w.logits = (float*)take((size_t)(T * E) * 4);
+    w.topk_idx = (int32_t*)take(R * 4);
+    w.topk_w = (float*)take(R * 4);
+    w.n_groups = (int32_t*)take(16);
+    w.groups = (int32_t*)take(R * 12);
+    w.perm_t = (int32_t*)take(R * 4);
+    w.perm_j = (int32_t*)take(R * 4);
+    w.cnt = (int32_t*)take((size_t)(T * (H / 128)) * 4);
+    w.a = take(R * (size_t)I * 2);
+    w.d = (float*)take(R * (size_t)H * 4);
+    w.bytes = off;
+    return w;
+}
+
+static bool moe_decode_shape_ok(int64_t T, int64_t H, int64_t I, int32_t E, int32_t k) {
+    return T >= 1 && T <= 32 && E >= 1 && E <= 1024 && k >= 1 && k <= 32 && k <= E && H >= 256 && H % 256 == 0 &&
+           I >= 256 && I % 256 == 0 && H <= 65536 && I <= 65536 && (int64_t)E * 2 * I < ((int64_t)1 << 31) &&
+           (int64_t)E * H < ((int64_t)1 << 31) && moe_decode_smem_bytes(H, I) <= 227 * 1024;
+}
+
+size_t moe_layer_decode_workspace(int64_t T, int64_t H, int64_t I, int32_t E, int32_t k) {
+    if (!moe_decode_shape_ok(T, H, I, E, k)) return 0;
+    return moe_decode_ws(nullptr, T, H, I, E, k).bytes;
+}
+
+int moe_layer_decode(const void* h, const void* w_router, const float* logit_bias, int64_t T, int64_t H, int32_t E,
+                     int32_t k, const uint8_t* gu_codes, const uint8_t* gu_scales, const float* gu_gs, int64_t I,
+                     const uint8_t* dn_codes, const uint8_t* dn_scales, const float* dn_gs, float* logits_out,
+                     int32_t* topk_idx, float* topk_w, void* a_out, void* y, int y_dtype, void* ws, size_t ws_bytes,
+                     void* stream) {
+    if (!h || !w_router || !gu_codes || !gu_scales || !gu_gs || !dn_codes || !dn_scales || !dn_gs || !y)
+        return NVFP4_ERR_NULL;
+    if (!dtype_ok(y_dtype)) return NVFP4_ERR_DTYPE;
+    if (!moe_decode_shape_ok(T, H, I, E, k)) return NVFP4_ERR_SHAPE;
+    if (!aligned16(h) || !aligned16(w_router) || !aligned16(gu_codes) || !aligned16(gu_scales) ||
+        !aligned16(dn_codes) || !aligned16(dn_scales) || !aligned16(y) || !aligned16(a_out) ||
+        !aligned16(logits_out))
+        return NVFP4_ERR_ALIGN;
+    const MoeDecodeWs need = moe_decode_ws(nullptr, T, H, I, E, k);
+    if (!ws || ws_bytes < need.bytes) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NVFP4_ERR_ALIGN;
+    NVFP4_TRY(check_arch());
+    const MoeDecodeWs w = moe_decode_ws(ws, T, H, I, E, k);
+    MoeDecodeLaunch L{};
+    L.h = h;
+    L.w_router = w_router;
+    L.logit_bias = logit_bias;
+    L.T = (int)T;
+    L.H = (int)H;
+    L.I = (int)I;
+    L.E = E;
+    L.k = k;
+    L.gu_codes = gu_codes;
+    L.gu_scales = gu_scales;
+    L.gu_gs = gu_gs;
+    L.dn_codes = dn_codes;
+    L.dn_scales = dn_scales;
+    L.dn_gs = dn_gs;
+    L.logits = logits_out ? logits_out : w.logits;
+    L.topk_idx = topk_idx ? topk_idx : w.topk_idx;
+    L.topk_w = topk_w ? topk_w : w.topk_w;
+    L.n_groups = w.n_groups;
+    L.groups = w.groups;
+    L.perm_t = w.perm_t;
+    L.perm_j = w.perm_j;
+    L.cnt = w.cnt;
+    L.a = a_out ? a_out : w.a;
+    L.d = w.d;
+    L.y = y;
+    L.y_dtype = y_dtype;
+    L.status = device_status_ptr();
+    return launch_moe_decode(L, (cudaStream_t)stream);
+}
+
 // ---- MoE grouped linear ------------------------------------------------------------
 
 static int resolve_grouped_mode(int mode, int64_t R) {
@@ -355,6 +453,25 @@ size_t moe_grouped_linear_workspace(int64_t R, int64_t K, int64_t N, int32_t E, 
     }
     if (mode == NVFP4_MODE_W4A4) need += grouped_w4a4_ws(nullptr, R, K, N, E, k, epilogue).bytes;
     return need;
+}
+
+int moe_grouped_linear_w4a4_ws_layout(int64_t R, int64_t K, int64_t N, int32_t E, int32_t k, int epilogue,
+                                      int64_t* out) {
+    if (!out) return NVFP4_ERR_NULL;
+    if (epilogue != NVFP4_EPI_NONE && epilogue != NVFP4_EPI_SWIGLU && epilogue != NVFP4_EPI_COMBINE)
+        return NVFP4_ERR_MODE;
+    if (E < 1 || E > 1024 || R < 1 || R > ((int64_t)1 << 26) || N < 1 || N > ((int64_t)1 << 20) || K < 256 ||
+        K % 256 || K > ((int64_t)1 << 20))
+        return NVFP4_ERR_SHAPE;
+    char* base = (char*)(uintptr_t)4096;  // offsets only: the layout from a stand-in base
+    const GroupedW4A4Ws o = grouped_w4a4_ws(base, R, K, N, E, k, epilogue);
+    out[0] = (char*)o.gs_x - base;
+    out[1] = (char*)o.pad_off - base;
+    out[2] = (char*)o.src_rows - base;
+    out[3] = (char*)o.codes - base;
+    out[4] = (char*)o.scales - base;
+    out[5] = moe_w4a4_rows(R, E);
+    return NVFP4_OK;
 }
 
 int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const int32_t* expert_offsets,
@@ -402,19 +519,14 @@ int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const 
                                   w.scales, w.gs_x, st, w.pad_off + E));
         const int64_t sf_stride = (int64_t)scales_bytes(N, K, NVFP4_SF_TILED);
         if (epilogue == NVFP4_EPI_COMBINE) {
-            const int64_t T = R / k;
-            float* acc = y_dtype == NVFP4_DTYPE_F32 ? (float*)y : w.yacc;
-            if (cudaMemsetAsync(acc, 0, (size_t)(T * N) * 4, st) != cudaSuccess) return NVFP4_ERR_LAUNCH;
-            NVFP4_TRY(launch_row_token(row_of, topk_w, R, k, w.tok_of, w.w_of, st));
+            // the experts' rows in bf16, then the weighted sum in slot order
             NVFP4_TRY(launch_gemm_w4a4_grouped(w.codes, w.scales, w.gs_x, rp, K, w.tile_info, w_codes, w_scales,
-                                               sf_stride, w_gs, E, N, epilogue, nullptr, NVFP4_DTYPE_F32, acc,
-                                               w.tok_of, w.w_of, device_status_ptr(), st));
-            if (y_dtype == NVFP4_DTYPE_BF16) return launch_f32_to_bf16(acc, T * N, y, st);
-            return NVFP4_OK;
+                                               sf_stride, w_gs, E, N, NVFP4_EPI_NONE, w.d, NVFP4_DTYPE_BF16,
+                                               device_status_ptr(), st));
+            return launch_combine(w.d, NVFP4_DTYPE_BF16, topk_w, row_of, R / k, k, N, y, y_dtype, st);
         }
         return launch_gemm_w4a4_grouped(w.codes, w.scales, w.gs_x, rp, K, w.tile_info, w_codes, w_scales, sf_stride,
-                                        w_gs, E, N, epilogue, y, y_dtype, nullptr, nullptr, nullptr,
-                                        device_status_ptr(), st);
+                                        w_gs, E, N, epilogue, y, y_dtype, device_status_ptr(), st);
     }
     char* wp = (char*)ws;
     float* d = nullptr;
@@ -450,7 +562,7 @@ int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const 
         a.y_dtype = NVFP4_DTYPE_F32;
         a.ldy = N;
         NVFP4_TRY(launch_gemv_w4a16(a, st));
-        return launch_combine(d, topk_w, row_of, R / k, k, N, y, y_dtype, st);
+        return launch_combine(d, NVFP4_DTYPE_F32, topk_w, row_of, R / k, k, N, y, y_dtype, st);
     }
     a.epilogue = epilogue;
     a.y = y;

@@ -34,8 +34,8 @@
 // the stacked [E * N, K/2] codes and the expert's scale block and gs.
 // Epilogues: NONE (y = acc * g); SWIGLU (gate tile = rows j0.. of the expert,
 // up tile = rows N/2 + j0..: two N = 128 MMAs into two accumulators, then
-// y = silu(g) * u); COMBINE (y[token] += topk_w * acc with fp32 vector
-// reductions; y is zeroed first).
+// y = silu(g) * u).  The weighted combine of the experts' rows runs after the
+// GEMM, as a gather in slot order (moe.cu), so its sums are deterministic.
 #include <cuda.h>
 
 #include <mutex>
@@ -70,9 +70,6 @@ struct GemmArgs {
     const int32_t* tile_info;  // grouped: per 128-row tile {expert, first output row, real rows}
     void* y;
     int64_t ldy;
-    float* yacc;               // COMBINE: fp32 [T, N] accumulation target
-    const int32_t* tok_of;     // COMBINE: token of each permuted row
-    const float* w_of;         // COMBINE: routing weight of each permuted row
     int* status;
 };
 
@@ -236,19 +233,7 @@ __global__ void __launch_bounds__(w4a4::kThreads, 1)
             const float4 v = *reinterpret_cast<const float4*>(so + rr * kOutStride + 4 * lane);
             const float vv[4] = {v.x, v.y, v.z, v.w};
             const int64_t orow = out_row0 + rr;
-            if constexpr (EPI == NVFP4_EPI_COMBINE) {
-                const int64_t tok = a.tok_of[orow];
-                const float wgt = a.w_of[orow];
-                float* yr = a.yacc + tok * a.ldy + col;
-                if (col + 4 <= ncols && (a.ldy & 3) == 0) {
-                    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(yr), "f"(wgt * v.x),
-                                 "f"(wgt * v.y), "f"(wgt * v.z), "f"(wgt * v.w)
-                                 : "memory");
-                } else {
-                    for (int t = 0; t < 4; ++t)
-                        if (col + t < ncols) atomicAdd(yr + t, wgt * vv[t]);
-                }
-            } else {
+            {
                 OutT* yp = reinterpret_cast<OutT*>(a.y) + orow * a.ldy + col;
                 if (col + 4 <= ncols && (a.ldy & 3) == 0) {
                     if constexpr (sizeof(OutT) == 4) {
@@ -315,8 +300,7 @@ int launch_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales, const floa
 int launch_gemm_w4a4_grouped(const uint8_t* a_codes, const uint8_t* a_scales, const float* gs_a, int64_t rows_pad,
                              int64_t K, const int32_t* tile_info, const uint8_t* w_codes, const uint8_t* w_scales,
                              int64_t sf_stride, const float* w_gs, int32_t E, int64_t N, int epilogue, void* y,
-                             int y_dtype, float* yacc, const int32_t* tok_of, const float* w_of, int* status,
-                             cudaStream_t st) {
+                             int y_dtype, int* status, cudaStream_t st) {
     CUtensorMap ma, mb;
     if (!make_tmap_2d_u8(&ma, a_codes, (uint64_t)(K / 2), (uint64_t)rows_pad, 128, w4a4::BM, 1)) return NVFP4_ERR_LAUNCH;
     if (!make_tmap_2d_u8(&mb, w_codes, (uint64_t)(K / 2), (uint64_t)E * (uint64_t)N, 128, w4a4::BN, 1))
@@ -332,19 +316,12 @@ int launch_gemm_w4a4_grouped(const uint8_t* a_codes, const uint8_t* a_scales, co
     a.gs_b = w_gs;
     a.tile_info = tile_info;
     a.y = y;
-    a.yacc = yacc;
-    a.tok_of = tok_of;
-    a.w_of = w_of;
     a.status = status;
     const int64_t mt = rows_pad / w4a4::BM;
     if (epilogue == NVFP4_EPI_SWIGLU) {
         a.ldy = N / 2;
         if (y_dtype == NVFP4_DTYPE_BF16) return launch_typed<__nv_bfloat16, NVFP4_EPI_SWIGLU, true>(ma, mb, a, mt, st);
         return launch_typed<float, NVFP4_EPI_SWIGLU, true>(ma, mb, a, mt, st);
-    }
-    if (epilogue == NVFP4_EPI_COMBINE) {
-        a.ldy = N;
-        return launch_typed<float, NVFP4_EPI_COMBINE, true>(ma, mb, a, mt, st);
     }
     a.ldy = N;
     if (y_dtype == NVFP4_DTYPE_BF16) return launch_typed<__nv_bfloat16, NVFP4_EPI_NONE, true>(ma, mb, a, mt, st);

@@ -363,7 +363,7 @@ static int launch_one(const DecodeArgs& a, const CUtensorMap& cm, const CUtensor
     attr[0].val.clusterDim.z = 1;
     set_pdl_attr(attr[1]);
     cfg.attrs = attr;
-    cfg.numAttrs = pdl_enabled() ? 2 : 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, cm, sm, a) == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 

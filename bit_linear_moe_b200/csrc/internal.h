@@ -8,9 +8,7 @@
 namespace nvfp4 {
 
 // Launch attribute for programmatic dependent launch (kernels that call
-// griddep_wait() before touching activations or outputs).  Off when the
-// environment sets NVFP4_PDL=0.
-bool pdl_enabled();
+// griddep_wait() before touching activations or outputs).
 inline void set_pdl_attr(cudaLaunchAttribute& a) {
     a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
     a.val.programmaticStreamSerializationAllowed = 1;
@@ -90,26 +88,55 @@ int launch_perm_scan(const int32_t* blk_counts, int64_t nblk, int32_t E, int32_t
                      cudaStream_t st);
 int launch_perm_scatter(const int32_t* topk_idx, int64_t T, int32_t E, int32_t k, const int32_t* blk_base,
                         int32_t* perm_tok, int32_t* perm_slot, int32_t* row_of, cudaStream_t st);
-int launch_combine(const float* d, const float* topk_w, const int32_t* row_of, int64_t T, int32_t k, int64_t N,
-                   void* y, int y_dtype, cudaStream_t st);
+// y[t] = sum_{j<k} topk_w[t, j] * d[row_of[t, j]], j ascending, fp32; d [T*k, N] in d_dtype; N % 4 == 0.
+int launch_combine(const void* d, int d_dtype, const float* topk_w, const int32_t* row_of, int64_t T, int32_t k,
+                   int64_t N, void* y, int y_dtype, cudaStream_t st);
 
 // Padded expert layout (rows_pad = multiple of 128 >= R + 127 E): pad_off[E+1],
 // tile_info[3 * rows_pad/128], src_rows[rows_pad].
 int launch_moe_pad(const int32_t* offsets, int32_t E, int64_t rows_pad, const int32_t* gather, int32_t* pad_off,
                    int32_t* tile_info, int32_t* src_rows, cudaStream_t st);
-int launch_f32_to_bf16(const float* src, int64_t n, void* dst, cudaStream_t st);  // n % 4 == 0
-// tok_of[row_of[i]] = i / k, w_of[row_of[i]] = topk_w[i] for i < n (= T * k).
 // experts with rows, compacted: list[j] for j < nslots (-1 past the last), E <= 1024.
 int launch_touched_experts(const int32_t* offsets, int32_t E, int32_t nslots, int32_t* list, cudaStream_t st);
-int launch_row_token(const int32_t* row_of, const float* topk_w, int64_t n, int32_t k, int32_t* tok_of, float* w_of,
-                     cudaStream_t st);
 
 // gemm_w4a4.cu, grouped: A = padded permuted activations, B = stacked experts.
 int launch_gemm_w4a4_grouped(const uint8_t* a_codes, const uint8_t* a_scales, const float* gs_a, int64_t rows_pad,
                              int64_t K, const int32_t* tile_info, const uint8_t* w_codes, const uint8_t* w_scales,
                              int64_t sf_stride, const float* w_gs, int32_t E, int64_t N, int epilogue, void* y,
-                             int y_dtype, float* yacc, const int32_t* tok_of, const float* w_of, int* status,
-                             cudaStream_t st);
+                             int y_dtype, int* status, cudaStream_t st);
+
+// moe_decode.cu: one routed expert layer for T <= 32 tokens (router, top-k,
+// gate/up + SwiGLU, down + combine), four kernels chained by PDL.
+struct MoeDecodeLaunch {
+    const void* h;              // [T, H] bf16
+    const void* w_router;       // [E, H] bf16
+    const float* logit_bias;    // [E] or null
+    int T, H, I, E, k;
+    const uint8_t* gu_codes;    // [E, 2I, H/2]
+    const uint8_t* gu_scales;   // E TILED blocks
+    const float* gu_gs;         // [E]
+    const uint8_t* dn_codes;    // [E, H, I/2]
+    const uint8_t* dn_scales;
+    const float* dn_gs;
+    float* logits;              // [T, E]
+    int32_t* topk_idx;          // [T, k]
+    float* topk_w;              // [T, k]
+    int32_t* n_groups;          // routing tables: [1]
+    int32_t* groups;            // [T * k][3]
+    int32_t* perm_t;            // [T * k]
+    int32_t* perm_j;            // [T * k]
+    int32_t* cnt;               // [T][H / 128]
+    void* a;                    // [T * k, I] bf16
+    float* d;                   // [T * k, H]
+    void* y;                    // [T, H]
+    int y_dtype;
+    int* status;
+};
+size_t moe_decode_smem_bytes(int64_t H, int64_t I);
+int launch_moe_decode(const MoeDecodeLaunch& L, cudaStream_t st);
+// the small-batch router kernel as a programmatic dependent launch
+int launch_router_logits_small_pdl(const void* h, const void* wr, const float* bias, int64_t T, int64_t H,
+                                   int32_t E, float* logits, cudaStream_t st);
 
 // Tokens per block of the routing permutation (top-k, counts, scatter): 32
 // gives one CTA per 32 tokens, so a 4,096-token batch spreads over 128 SMs.

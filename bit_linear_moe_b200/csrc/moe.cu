@@ -15,6 +15,8 @@
 // Combine        y[t, n] = sum_j w[t, j] * d[row_of[t, j], n], j ascending.
 #include "common.cuh"
 #include "internal.h"
+#include "tma.cuh"
+#include "topk.cuh"
 
 namespace nvfp4 {
 
@@ -93,6 +95,10 @@ __global__ void __launch_bounds__(256) router_logits_small_kernel(const __nv_bfl
     const int lane = threadIdx.x & 31;
     const int64_t gw = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);  // global warp
     const int64_t ngroups = (T + kRouterTokGroup - 1) / kRouterTokGroup;
+    // as a programmatic dependent: the next kernel may launch at once; the
+    // hidden states (written by the kernel before) are read after the wait
+    griddep_launch_dependents();
+    griddep_wait();
     if (gw >= (int64_t)E * ngroups) return;
     const int64_t e = gw / ngroups, t0 = (gw % ngroups) * kRouterTokGroup;
     const int nt = (int)((T - t0) < kRouterTokGroup ? (T - t0) : kRouterTokGroup);
@@ -120,6 +126,23 @@ __global__ void __launch_bounds__(256) router_logits_small_kernel(const __nv_bfl
     }
 }
 
+int launch_router_logits_small_pdl(const void* h, const void* wr, const float* bias, int64_t T, int64_t H,
+                                   int32_t E, float* logits, cudaStream_t st) {
+    const int64_t warps = (int64_t)E * ((T + kRouterTokGroup - 1) / kRouterTokGroup);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((warps + 7) / 8), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    set_pdl_attr(attr[0]);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, router_logits_small_kernel, (const __nv_bfloat16*)h, (const __nv_bfloat16*)wr,
+                              bias, T, H, E, logits) == cudaSuccess
+               ? NVFP4_OK
+               : NVFP4_ERR_LAUNCH;
+}
+
 int launch_router_logits(const void* h, const void* wr, const float* bias, int64_t T, int64_t H, int32_t E,
                          float* logits, cudaStream_t st) {
     if (T <= 64 && H % 8 == 0) {
@@ -138,12 +161,8 @@ int launch_router_logits(const void* h, const void* wr, const float* bias, int64
 
 // ---- top-k + per-block expert counts ------------------------------------
 // CTA = 1024 threads = 32 warps, kPermBlockTokens tokens; a warp takes
-// kPermBlockTokens / 32 of them.  Lane l holds logits l, l + 32, ... (PER of them) and keeps the best
-// of its untaken ones; a round is a warp arg-max over the lanes' bests, after
-// which only the winning lane rescans its own values.
+// kPermBlockTokens / 32 of them (warp_topk, topk.cuh).
 constexpr int kMaxE = 1024, kTopkThreads = 1024;
-
-NVFP4_DEV bool better(float v, int i, float bv, int bi) { return v > bv || (v == bv && i < bi); }
 
 template <int PER>
 __global__ void __launch_bounds__(kTopkThreads) topk_count_kernel(const float* __restrict__ logits, int64_t T,
@@ -158,51 +177,12 @@ __global__ void __launch_bounds__(kTopkThreads) topk_count_kernel(const float* _
     for (int tt = warp; tt < kPermBlockTokens; tt += kTopkThreads / 32) {
         const int64_t t = tb + tt;
         if (t >= T) break;
-        float v[PER];
-#pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            const int e = i * 32 + lane;
-            v[i] = e < E ? logits[t * E + e] : -INFINITY;
-        }
-        uint32_t taken = 0;  // bit i: v[i] already selected
-        auto rescan = [&](float& lbv, int& lbi) {
-            lbv = -INFINITY;
-            lbi = 0x7fffffff;
-#pragma unroll
-            for (int i = 0; i < PER; ++i) {
-                const int e = i * 32 + lane;
-                if (e < E && !((taken >> i) & 1u) && better(v[i], e, lbv, lbi)) {
-                    lbv = v[i];
-                    lbi = e;
-                }
-            }
-        };
-        float lbv;
-        int lbi;
-        rescan(lbv, lbi);
-        float lmax = 0.0f, mywl = 0.0f;
-        int myidx = 0;
-        for (int j = 0; j < k; ++j) {
-            float bv = lbv;
-            int bi = lbi;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-            }
-            if ((bi & 31) == lane) {
-                taken |= 1u << (bi >> 5);
-                rescan(lbv, lbi);
-            }
-            if (j == 0) lmax = bv;
-            if (lane == j) { myidx = bi; mywl = bv; }
-        }
-        const float ex = lane < k ? expf(mywl - lmax) : 0.0f;
-        const float den = warp_sum(ex);
+        int myidx;
+        float myw;
+        warp_topk<PER>(logits + t * E, E, k, lane, &myidx, &myw);
         if (lane < k) {
             topk_idx[t * k + lane] = myidx;
-            topk_w[t * k + lane] = ex / den;
+            topk_w[t * k + lane] = myw;
             atomicOr(&mask[myidx][tt >> 5], 1u << (tt & 31));
         }
     }
@@ -311,8 +291,22 @@ int launch_perm_scatter(const int32_t* topk_idx, int64_t T, int32_t E, int32_t k
 }
 
 // ---- combine ---------------------------------------------------------------
-template <typename OutT>
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ d, const float* __restrict__ w,
+// One thread per 4 output columns of a token: the k slots are read in order
+// j = 0..k-1 and summed in fp32, so the result does not depend on scheduling.
+template <typename InT>
+NVFP4_DEV float4 load4(const InT* p);
+template <>
+NVFP4_DEV float4 load4<float>(const float* p) {
+    return *reinterpret_cast<const float4*>(p);
+}
+template <>
+NVFP4_DEV float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    return make_float4(bf16lo_to_f32(u.x), bf16hi_to_f32(u.x), bf16lo_to_f32(u.y), bf16hi_to_f32(u.y));
+}
+
+template <typename InT, typename OutT>
+__global__ void __launch_bounds__(256) combine_kernel(const InT* __restrict__ d, const float* __restrict__ w,
                                                       const int32_t* __restrict__ row_of, int64_t T, int32_t k,
                                                       int64_t N, OutT* __restrict__ y) {
     const int64_t n4 = N / 4;
@@ -324,26 +318,36 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
         const float wj = w[t * k + j];
         const int32_t r = row_of[t * k + j];
         if (r < 0 || (int64_t)r >= T * k) continue;  // row_of must index the T * k rows of d
-        const float4 v = *reinterpret_cast<const float4*>(d + (int64_t)r * N + c);
+        const float4 v = load4<InT>(d + (int64_t)r * N + c);
         acc.x = fmaf(wj, v.x, acc.x);
         acc.y = fmaf(wj, v.y, acc.y);
         acc.z = fmaf(wj, v.z, acc.z);
         acc.w = fmaf(wj, v.w, acc.w);
     }
-    store_out<OutT>(y + t * N + c, acc.x);
-    store_out<OutT>(y + t * N + c + 1, acc.y);
-    store_out<OutT>(y + t * N + c + 2, acc.z);
-    store_out<OutT>(y + t * N + c + 3, acc.w);
+    if constexpr (sizeof(OutT) == 4) {
+        *reinterpret_cast<float4*>(y + t * N + c) = acc;
+    } else {
+        const __nv_bfloat162 b0 = __floats2bfloat162_rn(acc.x, acc.y);
+        const __nv_bfloat162 b1 = __floats2bfloat162_rn(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(y + t * N + c) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+    }
 }
 
-int launch_combine(const float* d, const float* topk_w, const int32_t* row_of, int64_t T, int32_t k, int64_t N,
-                   void* y, int y_dtype, cudaStream_t st) {
+int launch_combine(const void* d, int d_dtype, const float* topk_w, const int32_t* row_of, int64_t T, int32_t k,
+                   int64_t N, void* y, int y_dtype, cudaStream_t st) {
     const int64_t n = T * (N / 4);
     const unsigned grid = (unsigned)((n + 255) / 256);
-    if (y_dtype == NVFP4_DTYPE_BF16)
-        combine_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(d, topk_w, row_of, T, k, N, (__nv_bfloat16*)y);
-    else
-        combine_kernel<float><<<grid, 256, 0, st>>>(d, topk_w, row_of, T, k, N, (float*)y);
+#define NVFP4_C(IT, OT) \
+    combine_kernel<IT, OT><<<grid, 256, 0, st>>>((const IT*)d, topk_w, row_of, T, k, N, (OT*)y)
+    if (d_dtype == NVFP4_DTYPE_BF16) {
+        if (y_dtype == NVFP4_DTYPE_BF16) NVFP4_C(__nv_bfloat16, __nv_bfloat16);
+        else NVFP4_C(__nv_bfloat16, float);
+    } else {
+        if (y_dtype == NVFP4_DTYPE_BF16) NVFP4_C(float, __nv_bfloat16);
+        else NVFP4_C(float, float);
+    }
+#undef NVFP4_C
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 
@@ -414,48 +418,12 @@ __global__ void __launch_bounds__(256) moe_src_rows_kernel(const int32_t* __rest
     src_rows[pr] = src;
 }
 
-__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restrict__ src, int64_t n4,
-                                                          __nv_bfloat16* __restrict__ dst) {
-    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (i >= n4) return;
-    const float4 v = reinterpret_cast<const float4*>(src)[i];
-    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
-    uint2 o;
-    o.x = *reinterpret_cast<const uint32_t*>(&a);
-    o.y = *reinterpret_cast<const uint32_t*>(&b);
-    reinterpret_cast<uint2*>(dst)[i] = o;
-}
-
-// Inverse of row_of for the combine epilogue: tok_of[row] = token, w_of[row] = its routing weight.
-__global__ void __launch_bounds__(256) row_token_kernel(const int32_t* __restrict__ row_of,
-                                                        const float* __restrict__ topk_w, int64_t n, int32_t k,
-                                                        int32_t* __restrict__ tok_of, float* __restrict__ w_of) {
-    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (i >= n) return;
-    const int32_t r = row_of[i];
-    if (r < 0 || (int64_t)r >= n) return;  // row_of must be a permutation of [0, n)
-    tok_of[r] = (int32_t)(i / k);
-    w_of[r] = topk_w[i];
-}
-
-int launch_row_token(const int32_t* row_of, const float* topk_w, int64_t n, int32_t k, int32_t* tok_of, float* w_of,
-                     cudaStream_t st) {
-    row_token_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(row_of, topk_w, n, k, tok_of, w_of);
-    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
-}
-
 int launch_moe_pad(const int32_t* offsets, int32_t E, int64_t rows_pad, const int32_t* gather, int32_t* pad_off,
                    int32_t* tile_info, int32_t* src_rows, cudaStream_t st) {
     moe_pad_kernel<<<1, kMaxE, 0, st>>>(offsets, E, rows_pad / 128, pad_off, tile_info);
     if (cudaGetLastError() != cudaSuccess) return NVFP4_ERR_LAUNCH;
     moe_src_rows_kernel<<<(unsigned)((rows_pad + 255) / 256), 256, 0, st>>>(pad_off, offsets, E, gather, rows_pad,
                                                                             src_rows);
-    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
-}
-
-int launch_f32_to_bf16(const float* src, int64_t n, void* dst, cudaStream_t st) {
-    const int64_t n4 = n / 4;
-    f32_to_bf16_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, st>>>(src, n4, (__nv_bfloat16*)dst);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 

@@ -15,6 +15,8 @@
 // other threads) race on it and must be serialized by the caller.
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -30,17 +32,23 @@ size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
 // array's name is only a host-side stand-in; the real address comes from
 // cudaGetSymbolAddress, made once per device with that device current (the
 // first call on a device does it, so that call should come before any stream
-// capture).
+// capture).  The slots are atomic, so host threads making their first calls
+// at the same time are safe (each stores the same address).  The cached
+// address belongs to the device's primary context: after a device reset
+// (cudaDeviceReset) it is stale, and this entry point must not be called again
+// in that process.
 unsigned char* scratch_ptr() {
-    static unsigned char* cache[64] = {nullptr};
+    static std::atomic<unsigned char*> cache[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!cache[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return nullptr;
-        cache[dev] = (unsigned char*)p;
+    unsigned char* p = cache[dev].load(std::memory_order_acquire);
+    if (!p) {
+        void* q = nullptr;
+        if (cudaGetSymbolAddress(&q, g_route_scratch) != cudaSuccess) return nullptr;
+        p = (unsigned char*)q;
+        cache[dev].store(p, std::memory_order_release);
     }
-    return cache[dev];
+    return p;
 }
 
 }  // namespace

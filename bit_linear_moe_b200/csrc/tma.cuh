@@ -68,17 +68,21 @@ NVFP4_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete.
-NVFP4_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+// Bounded wait for the phase with the given parity to complete: false (and
+// NVFP4_ERR_DEVICE_TIMEOUT recorded in *status) after `limit` cycles.
+NVFP4_DEV bool mbar_wait_limit(uint64_t* bar, uint32_t parity, int* status, long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             if (status) atomicExch(status, NVFP4_ERR_DEVICE_TIMEOUT);
             return false;
         }
     }
     return true;
+}
+NVFP4_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+    return mbar_wait_limit(bar, parity, status, kWaitCycles);
 }
 
 // 2D tiled TMA load (no multicast) completing on `bar`.

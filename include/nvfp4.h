@@ -111,6 +111,15 @@ size_t nvfp4_scales_bytes(int64_t rows, int64_t cols, int sf_layout);
  * synchronizes `stream`.  The only call that synchronizes. */
 int nvfp4_read_device_status(void* stream, int* status_out);
 
+/* Debug helper for the bounded waits (Ignis README, "Credits": a per-request
+ * error boundary).  Launches one CTA that waits on an mbarrier nothing arrives
+ * on, with the bounded wait every TMA / tensor-core kernel here uses, limited
+ * to limit_cycles SM clock cycles (1 .. 4e9).  Nothing is in flight while it
+ * waits; when the limit runs out the kernel records NVFP4_ERR_DEVICE_TIMEOUT
+ * in the status word and returns, and the device stays usable.  Returns
+ * NVFP4_ERR_SHAPE for a limit out of range. */
+int nvfp4_debug_wait_timeout(int64_t limit_cycles, void* stream);
+
 /* ---- nvfp4_quantize ------------------------------------------------------
  * NVFP4 quantization (imp v0.20.0 release notes, "Highlights": first-party
  * NVFP4 quantizer, round-to-nearest part).  For x [rows, cols]:
@@ -156,6 +165,18 @@ int nvfp4_linear(const void* x, int x_dtype, int64_t M, int64_t K,
                  const float* w_gs, int64_t N,
                  void* y, int y_dtype, int mode,
                  void* ws, size_t ws_bytes, void* stream);
+
+/* ---- nvfp4_linear_w4a4_ws_layout -------------------------------------------
+ * Where a W4A4 nvfp4_linear call leaves the activations it quantized, inside
+ * its workspace: once the call has run (stream order), the bytes at these
+ * offsets from ws hold
+ *   offsets[0]  gs_x, one float (amax(|x|) / 2688, as nvfp4_quantize)
+ *   offsets[1]  codes [M, K/2]
+ *   offsets[2]  scales, TILED for M rows
+ * exactly what nvfp4_quantize(x, gs_in = NULL, TILED) writes, so a caller can
+ * hand them to nvfp4_linear_w4a4q for another weight with the same input.
+ * Requires K % 256 == 0, M >= 1. */
+int nvfp4_linear_w4a4_ws_layout(int64_t M, int64_t K, int64_t offsets[3]);
 
 /* ---- nvfp4_linear_w4a4q ---------------------------------------------------
  * The W4A4 linear with activations already in NVFP4 (e.g. written by a
@@ -226,7 +247,9 @@ int moe_route_topk(const void* h, const void* w_router, const float* logit_bias,
  * pieces), plus T * E * 4 bytes when logits_out is NULL; a request that does
  * not fit returns NVFP4_ERR_WORKSPACE before launching anything (pass
  * logits_out to route large T).  The first call on a device looks up the
- * array's device address, so make it before any stream capture.  Every call
+ * array's device address, so make it before any stream capture; the address
+ * stays cached for the process, so do not call this again after a device
+ * reset (cudaDeviceReset) in the same process.  Every call
  * shares the array: calls that overlap on the GPU race and must be
  * serialized by the caller.  Arguments, layouts and errors are otherwise
  * those of moe_route_topk. */
@@ -235,6 +258,42 @@ int moe_route_topk_noalloc(const void* h, const void* w_router, const float* log
                            float* logits_out, int32_t* topk_idx, float* topk_w,
                            int32_t* expert_offsets, int32_t* perm_tok, int32_t* perm_slot,
                            int32_t* row_of, void* stream);
+
+/* ---- moe_layer_decode ----------------------------------------------------
+ * One routed mixture-of-experts layer for a decode batch of T <= 32 tokens,
+ * from the router to the weighted combine, reading only the chosen experts'
+ * weights (CHImp Alpha v1.0 model card, "How it fits on one GPU": each token
+ * goes to 10 of 512 experts per layer and only those experts are read).
+ *     l[t, e]  = sum_h h[t, h] * Wr[e, h] (+ logit_bias[e]), fp32
+ *     topk_idx, topk_w as moe_route_topk (ties -> lower index; softmax over
+ *                the k selected)
+ *     a[t*k+j, c] = bf16(silu(g) * u), g = h[t] . Wgu[e][c],
+ *                u = h[t] . Wgu[e][I + c], e = topk_idx[t, j]   (W4A16)
+ *     y[t, n]  = sum_{j<k} topk_w[t, j] * (a[t*k+j] . Wd[e][n]), j ascending,
+ *                fp32 (the per-slot dot products are fp32; y rounded to
+ *                y_dtype at the end)
+ *   h          [T, H] bf16;  w_router [E, H] bf16;  logit_bias [E] or NULL
+ *   gu_codes   [E, 2I, H/2], gu_scales E consecutive TILED blocks of
+ *              nvfp4_scales_bytes(2I, H, TILED), gu_gs [E]  (rows 0..I-1 of an
+ *              expert are the gate projection, I..2I-1 the up projection)
+ *   dn_codes   [E, H, I/2], dn_scales E TILED blocks of
+ *              nvfp4_scales_bytes(H, I, TILED), dn_gs [E]
+ *   logits_out [T, E] fp32, topk_idx [T, k] int32, topk_w [T, k] fp32,
+ *   a_out      [T*k, I] bf16: optional outputs (NULL: kept in the workspace)
+ *   y          [T, H] in y_dtype (F32 or BF16)
+ *   ws         scratch of moe_layer_decode_workspace(T, H, I, E, k) bytes;
+ *              contents on entry are ignored.
+ * The layer runs as four kernels chained by programmatic dependent launch.
+ * Requires 1 <= T <= 32, 1 <= k <= 32, k <= E <= 1024, H % 256 == 0,
+ * I % 256 == 0, TILED scales; the workspace query returns 0 for shapes out
+ * of range. */
+size_t moe_layer_decode_workspace(int64_t T, int64_t H, int64_t I, int32_t E, int32_t k);
+int moe_layer_decode(const void* h, const void* w_router, const float* logit_bias,
+                     int64_t T, int64_t H, int32_t E, int32_t k,
+                     const uint8_t* gu_codes, const uint8_t* gu_scales, const float* gu_gs, int64_t I,
+                     const uint8_t* dn_codes, const uint8_t* dn_scales, const float* dn_gs,
+                     float* logits_out, int32_t* topk_idx, float* topk_w, void* a_out,
+                     void* y, int y_dtype, void* ws, size_t ws_bytes, void* stream);
 
 /* ---- moe_grouped_linear --------------------------------------------------
  * Expert linears over the permuted rows (CHImp, same section: only the chosen
@@ -246,15 +305,19 @@ int moe_route_topk_noalloc(const void* h, const void* w_router, const float* log
  *     SWIGLU   y[r, j]  = silu(out[r, j]) * out[r, N/2 + j]        y [R, N/2]
  *              (gate = first half of W_e's rows, up = second half)
  *     COMBINE  y[t, n]  = sum_{j<k} topk_w[t, j] * out[row_of[t, j], n],
- *              j ascending                                          y [R/k, N]
+ *              j ascending, fp32                                    y [R/k, N]
+ *              (W4A4 rounds out[r, :] to bf16 before the sum, the layer's
+ *              bf16 expert output; W4A16 keeps it fp32.  Either way the
+ *              sum is deterministic: the same inputs give the same bits.)
  *   x        [rows of x, K] bf16 (x_dtype BF16)
  *   w_codes  [E, N, K/2];  w_scales: E consecutive per-expert scale blocks of
  *            nvfp4_scales_bytes(N, K, w_sf_layout) bytes;  w_gs [E] fp32
  *   R        total rows (= T * k for routed input)
  *   topk_w, row_of, k: used by COMBINE only (may be NULL / 0 otherwise)
  *   y_dtype  F32 or BF16
- *   mode     as nvfp4_linear (W4A16 / W4A4 / AUTO by R <= 32 * k ... see
- *            moe_grouped_linear_workspace); W4A4 requires TILED scales.
+ *   mode     W4A16, W4A4, or AUTO: W4A16 if R <= 512, else W4A4.  W4A4
+ *            requires TILED scales, K % 256 == 0 and N % 128 == 0 (N % 256
+ *            for SWIGLU).
  *   ws       scratch of moe_grouped_linear_workspace(...) bytes.
  * Experts with no rows are skipped: their weights are not read. */
 size_t moe_grouped_linear_workspace(int64_t R, int64_t K, int64_t N, int32_t E, int32_t k,
@@ -267,6 +330,26 @@ int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather,
                        int epilogue, const float* topk_w, const int32_t* row_of, int32_t k,
                        void* y, int y_dtype, int mode,
                        void* ws, size_t ws_bytes, void* stream);
+
+/* ---- moe_grouped_linear_w4a4_ws_layout -------------------------------------
+ * Where a W4A4 moe_grouped_linear call leaves the permuted activations it
+ * quantized, inside its workspace.  Each expert's rows are padded to a whole
+ * number of 128-row tiles; once the call has run (stream order), the bytes at
+ * these offsets from ws hold
+ *   out[0]  gs_x, one float: amax over the rows read (x[perm_tok[r]] when
+ *           gathering, x[r] otherwise) / 2688
+ *   out[1]  pad_off int32 [E+1]: first padded row of each expert; pad_off[E]
+ *           is the number of padded rows in use
+ *   out[2]  src_rows int32 [out[5]]: the row of x each padded row quantizes,
+ *           -1 for padding
+ *   out[3]  codes [out[5], K/2] of the padded rows (padding rows are 0)
+ *   out[4]  scales, TILED for out[5] rows (padding rows are 0)
+ *   out[5]  the padded row count the workspace is laid out for
+ * Rows at or past pad_off[E] are not written.  Codes and scales of row pr
+ * equal those nvfp4_quantize gives row src_rows[pr] of x with gs_in = gs_x.
+ * Requires K % 256 == 0 and the other limits of moe_grouped_linear. */
+int moe_grouped_linear_w4a4_ws_layout(int64_t R, int64_t K, int64_t N, int32_t E, int32_t k, int epilogue,
+                                      int64_t out[6]);
 
 #ifdef __cplusplus
 }

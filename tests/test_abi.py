@@ -196,3 +196,51 @@ def test_noalloc_scratch_limit(L):
     if not torch.cuda.is_available():
         assert route(8192, FAKE) == nv.ERR_ARCH                 # fits: validation passes, then no B200
         assert route(32, None) == nv.ERR_ARCH
+
+
+def test_grouped_auto_mode_threshold(L):
+    """AUTO runs the grouped linear as W4A16 for R <= 512 rows and as W4A4 above:
+    the workspace query follows the same rule (k = 10, so the switch is not at
+    32 * k = 320 rows)."""
+    K, N, E, k = 2048, 1024, 512, 10
+    for epi in (nv.EPI_NONE, nv.EPI_SWIGLU, nv.EPI_COMBINE):
+        for R in (320, 321, 512, 513):
+            auto = L.moe_grouped_linear_workspace(R, K, N, E, k, epi, nv.MODE_AUTO)
+            want = nv.MODE_W4A16 if R <= 512 else nv.MODE_W4A4
+            assert auto == L.moe_grouped_linear_workspace(R, K, N, E, k, epi, want), (epi, R)
+        assert (L.moe_grouped_linear_workspace(512, K, N, E, k, epi, nv.MODE_W4A16)
+                != L.moe_grouped_linear_workspace(512, K, N, E, k, epi, nv.MODE_W4A4))
+
+
+def test_w4a4_workspace_layouts(L):
+    """The documented places of the quantized activations inside the W4A4
+    workspaces: inside the workspace the size query returns, 16-byte aligned,
+    in the stated order."""
+    M, K = 2048, 5120
+    lay = nv.nvfp4_linear_w4a4_ws_layout(M, K)
+    need = L.nvfp4_linear_workspace(M, K, 4096, nv.MODE_W4A4)
+    assert lay["gs_x"] % 4 == 0 and lay["codes"] % 16 == 0 and lay["scales"] % 16 == 0
+    assert lay["codes"] + M * K // 2 <= lay["scales"]
+    assert lay["scales"] + nv.nvfp4_scales_bytes(M, K, nv.SF_TILED) <= need
+    with pytest.raises(nv.NVFP4Error):
+        nv.nvfp4_linear_w4a4_ws_layout(M, 5000)
+    R, E, k, N = 40960, 512, 10, 1024
+    for epi in (nv.EPI_NONE, nv.EPI_SWIGLU, nv.EPI_COMBINE):
+        g = nv.moe_grouped_linear_w4a4_ws_layout(R, 2048, N, E, k, epi)
+        need = L.moe_grouped_linear_workspace(R, 2048, N, E, k, epi, nv.MODE_W4A4)
+        rp = g["rows_pad"]
+        assert rp % 128 == 0 and rp >= R + 127 * E
+        assert g["pad_off"] + 4 * (E + 1) <= g["src_rows"]
+        assert g["src_rows"] + 4 * rp <= g["codes"]
+        assert g["codes"] + rp * 1024 <= g["scales"]
+        assert g["scales"] + nv.nvfp4_scales_bytes(rp, 2048, nv.SF_TILED) <= need
+        assert all(v % 16 == 0 for key, v in g.items() if key != "rows_pad")
+    with pytest.raises(nv.NVFP4Error):
+        nv.moe_grouped_linear_w4a4_ws_layout(R, 2000, N, E, k, nv.EPI_NONE)
+
+
+def test_debug_wait_timeout_validation(L):
+    assert L.nvfp4_debug_wait_timeout(0, None) == nv.ERR_SHAPE
+    assert L.nvfp4_debug_wait_timeout(5_000_000_000, None) == nv.ERR_SHAPE
+    if not torch.cuda.is_available():
+        assert L.nvfp4_debug_wait_timeout(1000, None) == nv.ERR_ARCH

@@ -16,7 +16,8 @@ import bit_linear_moe_b200 as nv
 import oracle
 from oracle import moe as omoe
 from bit_linear_moe_b200 import synth
-from nvfp4_checks import assert_within_bound, bf16_ulp
+from moe_fixtures import moe512_q, quantize_experts, stack_tiled, swiglu_bound
+from nvfp4_checks import assert_within_bound, bf16_ulp, tiled_to_rowmajor
 
 pytestmark = pytest.mark.gpu
 E, H, I, K_TOP = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_K
@@ -205,83 +206,132 @@ def test_untouched_experts_are_not_read():
 
 # ---- grouped W4A4 (tensor-core) expert layer ---------------------------------
 
-def _w4a4_layer(E, T, zipf_like, seed=20):
-    """E experts with the per-expert shapes of the 512-expert layer; weights
-    quantized on the GPU (bit-exactness of that quantizer is tested in
-    test_gpu_quantize) and by the oracle for the experts it checks."""
-    rng = np.random.default_rng(seed)
-    wr = synth.to_bf16(0.02 * rng.standard_normal((E, H)))
-    h = synth.activations(np.random.default_rng([seed, T]), T, H)
-    bias = (-1.1 * np.log(np.random.default_rng([seed, 1]).permutation(E) + 1)).astype(np.float32) if zipf_like \
-        else None
-    gu_f = [synth.weight(np.random.default_rng([seed, 2, e]), 2 * I, H) for e in range(E)]
-    dn_f = [synth.weight(np.random.default_rng([seed, 3, e]), H, I) for e in range(E)]
-
-    def stack(ws):
-        N, K = ws[0].shape
-        sb = nv.nvfp4_scales_bytes(N, K, nv.SF_TILED)
-        codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device="cuda")
-        scales = torch.empty(E * sb, dtype=torch.uint8, device="cuda")
-        gs = torch.empty(E, dtype=torch.float32, device="cuda")
-        for e, w in enumerate(ws):
-            nv.nvfp4_quantize(torch.from_numpy(w).cuda(), sf_layout=nv.SF_TILED, codes=codes[e],
-                              scales=scales[e * sb:(e + 1) * sb], gs_out=gs[e:e + 1])
-        return codes, scales, gs
-
-    return h, wr, bias, gu_f, dn_f, stack(gu_f), stack(dn_f)
+def _grouped_ws_activations(ws, R, K, N, E_, epi):
+    lay = nv.moe_grouped_linear_w4a4_ws_layout(R, K, N, E_, K_TOP, epi)
+    b = ws.cpu().numpy()
+    rp = lay["rows_pad"]
+    gs = b[lay["gs_x"]:lay["gs_x"] + 4].view(np.float32)[0]
+    pad_off = b[lay["pad_off"]:lay["pad_off"] + 4 * (E_ + 1)].view(np.int32).copy()
+    src = b[lay["src_rows"]:lay["src_rows"] + 4 * rp].view(np.int32).copy()
+    codes = b[lay["codes"]:lay["codes"] + rp * K // 2].reshape(rp, K // 2).copy()
+    sc = tiled_to_rowmajor(b[lay["scales"]:lay["scales"] + nv.nvfp4_scales_bytes(rp, K, nv.SF_TILED)], rp, K)
+    return gs, pad_off, src, codes, sc
 
 
-@pytest.mark.parametrize("zipf", [False, True])
-def test_expert_layer_w4a4_4096_tokens(zipf):
-    E_, T = 64, 4096
-    h, wr, bias, gu_f, dn_f, (gc, gsc, ggs), (dc, dsc, dgs) = _w4a4_layer(E_, T, zipf)
+def _check_permuted_activations(ws, x_np, xd, R, K, N, E_, epi, off, perm_tok):
+    """The padded, permuted activations a grouped W4A4 call quantized: the row
+    map is each expert's rows padded to whole 128-row tiles; codes, scales and
+    gs equal the oracle's quantization of the gathered rows (bit-exact, every
+    row); and quantize(permute(x)) == permute(quantize(x)) on the GPU."""
+    gs, pad_off, src, codes, sc = _grouped_ws_activations(ws, R, K, N, E_, epi)
+    cnt = np.diff(off)
+    want_pad = np.concatenate([[0], np.cumsum((cnt + 127) // 128 * 128)]).astype(np.int32)
+    assert np.array_equal(pad_off, want_pad)
+    used = int(want_pad[-1])
+    want_src = np.full(used, -1, np.int32)
+    for e in np.flatnonzero(cnt):
+        rows = np.arange(off[e], off[e + 1])
+        want_src[want_pad[e]:want_pad[e] + cnt[e]] = perm_tok[rows] if perm_tok is not None else rows
+    assert np.array_equal(src[:used], want_src)
+    real = want_src >= 0
+    gathered = x_np[want_src[real]]
+    q = oracle.quantize(gathered, gs=oracle.global_scale(gathered))
+    assert gs == q[2], f"gs_x {gs!r} != {q[2]!r}"
+    assert np.array_equal(codes[:used][real], q[0]), f"{(codes[:used][real] != q[0]).sum()} code bytes differ"
+    assert np.array_equal(sc[:used][real], q[1]), f"{(sc[:used][real] != q[1]).sum()} scales differ"
+    assert not codes[:used][~real].any() and not sc[:used][~real].any(), "padding rows must be zero"
+    # the same identity on the GPU: the dense quantizer with the same gs, then the row map
+    gsd = torch.tensor([gs], dtype=torch.float32, device="cuda")
+    c_full, s_full, _ = nv.nvfp4_quantize(xd, gs_in=gsd, sf_layout=nv.SF_ROWMAJOR)
+    torch.cuda.synchronize()
+    c_full, s_full = c_full.cpu().numpy(), s_full.cpu().numpy().reshape(-1, K // 16)
+    assert np.array_equal(codes[:used][real], c_full[want_src[real]])
+    assert np.array_equal(sc[:used][real], s_full[want_src[real]])
+
+
+def _check_w4a4_layer(E_, T, h, wr, bias, gu_q, dn_q, ntok, seed):
+    """One W4A4 expert layer, stage by stage: the routed gate/up + SwiGLU, the
+    down projection (bf16 rows, the NONE epilogue) and the weighted combine,
+    each against the oracle on the GPU's own input to that stage; the permuted
+    activations of both projections bit-exact; the combine deterministic."""
+    R = T * K_TOP
+    gc, gsc, ggs = stack_tiled(gu_q)
+    dc, dsc, dgs = stack_tiled(dn_q)
     hd = torch.from_numpy(h).to(torch.bfloat16).cuda()
     out = nv.moe_route_topk(hd, torch.from_numpy(wr).to(torch.bfloat16).cuda(), K_TOP,
                             logit_bias=None if bias is None else torch.from_numpy(bias).cuda())
-    R = T * K_TOP
+    ws1 = torch.empty(int(nv.lib().moe_grouped_linear_workspace(R, H, 2 * I, E_, K_TOP, nv.EPI_SWIGLU,
+                                                                nv.MODE_W4A4)), dtype=torch.uint8, device="cuda")
     a = nv.moe_grouped_linear(hd, out["expert_offsets"], gc, gsc, ggs, R, perm_tok=out["perm_tok"], gather=True,
                               w_sf_layout=nv.SF_TILED, epilogue=nv.EPI_SWIGLU, y_dtype=torch.bfloat16,
-                              mode=nv.MODE_W4A4)
-    y = nv.moe_grouped_linear(a, out["expert_offsets"], dc, dsc, dgs, R, gather=False, w_sf_layout=nv.SF_TILED,
-                              epilogue=nv.EPI_COMBINE, topk_w=out["topk_w"], row_of=out["row_of"], k=K_TOP,
-                              y_dtype=torch.float32, mode=nv.MODE_W4A4)
+                              mode=nv.MODE_W4A4, ws=ws1)
+    ws2 = torch.empty(int(nv.lib().moe_grouped_linear_workspace(R, I, H, E_, K_TOP, nv.EPI_NONE, nv.MODE_W4A4)),
+                      dtype=torch.uint8, device="cuda")
+    d = nv.moe_grouped_linear(a, out["expert_offsets"], dc, dsc, dgs, R, gather=False, w_sf_layout=nv.SF_TILED,
+                              epilogue=nv.EPI_NONE, y_dtype=torch.bfloat16, mode=nv.MODE_W4A4, ws=ws2)
+    ys = [nv.moe_grouped_linear(a, out["expert_offsets"], dc, dsc, dgs, R, gather=False, w_sf_layout=nv.SF_TILED,
+                                epilogue=nv.EPI_COMBINE, topk_w=out["topk_w"], row_of=out["row_of"], k=K_TOP,
+                                y_dtype=torch.float32, mode=nv.MODE_W4A4) for _ in range(2)]
+    yb = nv.moe_grouped_linear(a, out["expert_offsets"], dc, dsc, dgs, R, gather=False, w_sf_layout=nv.SF_TILED,
+                               epilogue=nv.EPI_COMBINE, topk_w=out["topk_w"], row_of=out["row_of"], k=K_TOP,
+                               y_dtype=torch.bfloat16, mode=nv.MODE_W4A4)
     torch.cuda.synchronize()
     assert nv.nvfp4_read_device_status() == nv.OK
+    assert torch.equal(ys[0], ys[1]), "the combine is not bitwise reproducible"
+    assert torch.equal(yb, ys[0].to(torch.bfloat16)), "bf16 combine != bf16(fp32 combine)"
     g = {k2: v.cpu().numpy() for k2, v in out.items()}
-    a_np = a.float().cpu().numpy()
-    y_np = y.cpu().numpy()
     off, pt, row_of, tw = g["expert_offsets"], g["perm_tok"], g["row_of"], g["topk_w"].astype(np.float64)
+    a_np = a.float().cpu().numpy()
+    d_np = d.float().cpu().numpy()
+    y_np = ys[0].cpu().numpy()
+    _check_permuted_activations(ws1, h, hd, R, H, 2 * I, E_, nv.EPI_SWIGLU, off, pt)
+    _check_permuted_activations(ws2, a_np, a, R, I, H, E_, nv.EPI_NONE, off, None)
+    del ws1, ws2
+    # combine, every token, on the GPU's own bf16 expert rows
+    ref_y, ref_b = omoe.combine(d_np, tw, row_of)
+    assert_within_bound(y_np, ref_y, ref_b, False, "combine")
+    # gate/up + SwiGLU and down on the rows of `ntok` seeded tokens, grouped by expert
     expert_of_row = np.searchsorted(off, np.arange(R), side="right") - 1
-    toks = np.sort(np.random.default_rng(5).choice(T, 24, replace=False))
+    toks = np.sort(np.random.default_rng(seed).choice(T, ntok, replace=False))
+    rows = np.sort(row_of[toks].ravel())
     gs_h = oracle.global_scale(h)
     gs_a = oracle.global_scale(a_np)
-    q_gu, q_dn = {}, {}
-    for t in toks:
-        for j in range(K_TOP):
-            r = int(row_of[t, j])
-            e = int(expert_of_row[r])
-            if e not in q_gu:
-                q_gu[e] = oracle.quantize(gu_f[e])
-                q_dn[e] = oracle.quantize(dn_f[e])
-            # stage 1: gate/up (W4A4 on the gathered, quantized hidden state) + SwiGLU
-            xq = oracle.quantize(h[pt[r]:pt[r] + 1], gs=gs_h)
-            gu, gu_ad = oracle.linear_w4a4(xq, q_gu[e])
-            ref_a = omoe.swiglu(gu)[0]
-            gg, uu = gu[0, :I], gu[0, I:]
-            sig = 1.0 / (1.0 + np.exp(-gg))
-            dg, du = 1e-4 * gu_ad[0, :I] + 1e-6, 1e-4 * gu_ad[0, I:] + 1e-6
-            bound = (np.abs(uu) * np.abs(sig * (1 + gg * (1 - sig))) * dg + np.abs(gg * sig) * du + dg * du
-                     + 1e-5 * np.abs(ref_a) + 1e-6 + bf16_ulp(ref_a))
-            err = np.abs(a_np[r] - ref_a)
-            assert (err <= bound).all(), f"swiglu row {r}: max ratio {np.max(err / bound)}"
-        # stage 2: down projection of the GPU's own a, then the weighted combine
-        ref_y = np.zeros(H)
-        ref_b = np.zeros(H)
-        for j in range(K_TOP):
-            r = int(row_of[t, j])
-            e = int(expert_of_row[r])
-            aq = oracle.quantize(a_np[r:r + 1], gs=gs_a)
-            d, d_ad = oracle.linear_w4a4(aq, q_dn[e])
-            ref_y += tw[t, j] * d[0]
-            ref_b += abs(tw[t, j]) * d_ad[0]
-        assert_within_bound(y_np[t], ref_y, ref_b, False, f"down+combine token {t}")
+    for e in np.unique(expert_of_row[rows]):
+        re = rows[expert_of_row[rows] == e]
+        gu, gu_ad = oracle.linear_w4a4(oracle.quantize(h[pt[re]], gs=gs_h), gu_q[e])
+        ref_a = omoe.swiglu(gu)
+        err = np.abs(a_np[re] - ref_a)
+        bound = swiglu_bound(gu, gu_ad, ref_a)
+        assert (err <= bound).all(), f"swiglu expert {e}: max ratio {np.max(err / bound)}"
+        ref_d, d_ad = oracle.linear_w4a4(oracle.quantize(a_np[re], gs=gs_a), dn_q[e])
+        assert_within_bound(d_np[re], ref_d, d_ad, True, f"down expert {e}")
+    return int((np.diff(off) > 0).sum())
+
+
+@pytest.mark.parametrize("zipf", [False, True])
+def test_expert_layer_w4a4_64_experts(zipf):
+    """A 64-expert layer with the 512-expert layer's per-expert shapes: about
+    640 rows per expert, so most tiles are full."""
+    E_, T, seed = 64, 4096, 20
+    rng = np.random.default_rng(seed)
+    wr = synth.to_bf16(0.02 * rng.standard_normal((E_, H)))
+    h = synth.activations(np.random.default_rng([seed, T]), T, H)
+    bias = (-1.1 * np.log(np.random.default_rng([seed, 1]).permutation(E_) + 1)).astype(np.float32) if zipf \
+        else None
+    gu_q = quantize_experts([synth.weight(np.random.default_rng([seed, 2, e]), 2 * I, H) for e in range(E_)])
+    dn_q = quantize_experts([synth.weight(np.random.default_rng([seed, 3, e]), H, I) for e in range(E_)])
+    _check_w4a4_layer(E_, T, h, wr, bias, gu_q, dn_q, 64, 5)
+
+
+@pytest.mark.parametrize("zipf", [False, True])
+def test_expert_layer_w4a4_512_experts_4096_tokens(zipf):
+    """The 512-expert layer at 4,096 tokens (the W4A4 configuration): about 80
+    rows per expert under uniform routing, so every expert's tile is partial
+    and padding dominates; the Zipf run concentrates rows on a few experts.
+    256 seeded tokens (2,560 rows) are checked stage by stage."""
+    T = 4096
+    gu_q, dn_q = moe512_q()
+    h = synth.moe_hidden(T)
+    bias = synth.moe_zipf_bias() if zipf else None
+    touched = _check_w4a4_layer(E, T, h, _router(), bias, gu_q, dn_q, 256, 11)
+    print(f"E=512 T=4096 zipf={zipf}: {touched} experts touched")

@@ -17,7 +17,7 @@ import torch
 import bit_linear_moe_b200 as nv
 import oracle
 from bit_linear_moe_b200 import synth
-from nvfp4_checks import assert_within_bound, rowmajor_to_tiled
+from nvfp4_checks import assert_within_bound, rowmajor_to_tiled, tiled_to_rowmajor
 
 pytestmark = pytest.mark.gpu
 
@@ -67,35 +67,49 @@ def test_outlier_columns_small():
     assert_within_bound(y, ref, ad, False, "w4a4 outliers")
 
 
-@functools.lru_cache(maxsize=2)
+@functools.lru_cache(maxsize=1)
 def _dense_q(seed, K, N):
     return oracle.quantize(synth.dense_weight(seed, K, N))
 
 
+def _ws_activations(ws, M, K):
+    """The quantized activations a W4A4 nvfp4_linear call leaves in its workspace."""
+    lay = nv.nvfp4_linear_w4a4_ws_layout(M, K)
+    b = ws.cpu().numpy()
+    gs = b[lay["gs_x"]:lay["gs_x"] + 4].view(np.float32)[0]
+    codes = b[lay["codes"]:lay["codes"] + M * K // 2].reshape(M, K // 2)
+    sc = b[lay["scales"]:lay["scales"] + nv.nvfp4_scales_bytes(M, K, nv.SF_TILED)]
+    return gs, codes, tiled_to_rowmajor(sc, M, K)
+
+
+@pytest.mark.parametrize("M", synth.PREFILL_M)
 @pytest.mark.parametrize("name,K,N,seed", synth.DENSE27B)
-@pytest.mark.parametrize("M", [512, 2048])
-def test_prefill_shapes_sampled(name, K, N, seed, M):
+def test_prefill_shapes(name, K, N, seed, M):
+    """The prefill configurations on every 27B-shaped linear.  The activation
+    codes, scales and gs that nvfp4_linear quantizes into its workspace are
+    compared with the oracle's in full (bit-exact); the output on 256 seeded
+    rows x all N and on all M x 64 seeded columns."""
     wq = _dense_q(seed, K, N)
     x, _ = synth.prefill_x(seed, M, K)
-    y = _gpu(x, wq, torch.bfloat16)
+    c, s, g = _upload_w(wq, N, K)
+    xd = torch.from_numpy(x).to(torch.bfloat16).cuda()
+    ws = torch.empty(int(nv.lib().nvfp4_linear_workspace(M, K, N, nv.MODE_W4A4)), dtype=torch.uint8,
+                     device="cuda")
+    y = nv.nvfp4_linear(xd, c, s, g, w_sf_layout=nv.SF_TILED, y_dtype=torch.bfloat16, mode=nv.MODE_W4A4, ws=ws)
+    torch.cuda.synchronize()
+    assert nv.nvfp4_read_device_status() == nv.OK
+    del c, s, g, xd
+    gs_w, codes_w, sc_w = _ws_activations(ws, M, K)
+    del ws
+    xq = oracle.quantize(x)
+    assert gs_w == xq[2], f"{name} M={M}: gs_x {gs_w!r} != {xq[2]!r}"
+    assert np.array_equal(codes_w, xq[0]), f"{name} M={M}: {(codes_w != xq[0]).sum()} activation code bytes differ"
+    assert np.array_equal(sc_w, xq[1]), f"{name} M={M}: {(sc_w != xq[1]).sum()} activation scales differ"
+    y = y.float().cpu().numpy()
     rng = np.random.default_rng([seed, M, 7])
-    rows = np.sort(rng.choice(M, 16, replace=False))
+    rows = np.sort(rng.choice(M, min(M, 256), replace=False))
     cols = np.sort(rng.choice(N, 64, replace=False))
-    ref, ad = _ref(x, wq, rows=rows)
+    ref, ad = oracle.linear_w4a4((xq[0][rows], xq[1][rows], xq[2]), wq)
     assert_within_bound(y[rows], ref, ad, True, f"{name} M={M} sampled rows")
-    ref, ad = _ref(x, wq, cols=cols)
+    ref, ad = oracle.linear_w4a4(xq, (wq[0][cols], wq[1][cols], wq[2]))
     assert_within_bound(y[:, cols], ref, ad, True, f"{name} M={M} sampled cols")
-
-
-def test_prefill_8192_sampled():
-    name, K, N, seed = synth.DENSE27B[1]        # o_proj 5120 x 5120
-    wq = _dense_q(seed, K, N)
-    x, _ = synth.prefill_x(seed, 8192, K)
-    y = _gpu(x, wq, torch.bfloat16)
-    rng = np.random.default_rng(8192)
-    rows = np.sort(rng.choice(8192, 16, replace=False))
-    cols = np.sort(rng.choice(N, 16, replace=False))
-    ref, ad = _ref(x, wq, rows=rows)
-    assert_within_bound(y[rows], ref, ad, True, "M=8192 sampled rows")
-    ref, ad = _ref(x, wq, cols=cols)
-    assert_within_bound(y[:, cols], ref, ad, True, "M=8192 sampled cols")

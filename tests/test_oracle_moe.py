@@ -37,12 +37,40 @@ def test_topk_with_k_equal_E_is_full_softmax():
     assert np.allclose(np.take_along_axis(full, idx.astype(np.int64), axis=1), w, rtol=1e-12)
 
 
-def test_router_logits_match_library_matmul():
-    h = synth.moe_hidden(3)
-    wr = synth.moe_router()
-    bias = synth.moe_zipf_bias()
+def test_router_logits_hand_computed():
+    """l[t, e] = sum_h h[t, h] * Wr[e, h] + bias[e], worked by hand: a one-hot
+    token reads one column of Wr, a token of ones the row sums, and the bias is
+    added per expert (not per token).  A transposed Wr, a bias broadcast along
+    the wrong axis or a dropped bias gives other numbers."""
+    H, E = 4, 3
+    wr = np.array([[1.0, 2.0, 3.0, 4.0],
+                   [-1.0, 0.5, 0.0, 2.0],
+                   [0.25, 0.0, -2.0, 1.0]], dtype=np.float32)   # [E, H]
+    bias = np.array([10.0, 20.0, 30.0], dtype=np.float32)
+    h = np.array([[0.0, 1.0, 0.0, 0.0],                          # selects column 1 of Wr
+                  [1.0, 1.0, 1.0, 1.0],                          # row sums of Wr
+                  [2.0, 0.0, 0.0, -1.0]], dtype=np.float32)
     l = moe.router_logits(h, wr, bias)
-    assert np.allclose(l, h.astype(np.float64) @ wr.astype(np.float64).T + bias, rtol=1e-13, atol=1e-13)
+    expected = np.array([[2.0 + 10, 0.5 + 20, 0.0 + 30],
+                         [10.0 + 10, 1.5 + 20, -0.75 + 30],
+                         [-2.0 + 10, -4.0 + 20, -0.5 + 30]])
+    assert l.shape == (3, E)
+    assert np.array_equal(l, expected)
+    assert np.array_equal(moe.router_logits(h, wr), expected - bias[None, :].astype(np.float64))
+
+
+def test_router_logits_exact_in_fp64():
+    """bf16 x bf16 products have at most 16 significant bits, so at H = 2048 the
+    fp64 sum is exact: it equals the exact rational sum (brute force with
+    Fractions on a few tokens and experts)."""
+    from fractions import Fraction
+    h = synth.moe_hidden(2)
+    wr = synth.moe_router()
+    l = moe.router_logits(h, wr)
+    for t in range(2):
+        for e in (0, 17, 511):
+            exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(h[t], wr[e]))
+            assert Fraction(l[t, e]) == exact
 
 
 def test_zipf_bias_is_log_prior():
