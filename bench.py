@@ -512,6 +512,39 @@ def moe_section(nv, torch, dev, reps=30):
                                 "touched_experts_mean": round(sum(touched) / nbatch, 1),
                                 "GB/s": round(nbytes / (t * 1e-3) / 1e9, 1),
                                 "TFLOPs": round(flop / (t * 1e-3) / 1e12, 2)}
+    # the fused decode-time layer (router ... combine in one call) at T = 1, 32
+    for T, nbatch in ((1, 16), (32, 4)):
+        wsd = torch.empty(max(16, int(nv.lib().moe_layer_decode_workspace(T, H, I, E, k))), dtype=torch.uint8,
+                          device=dev)
+        for bias_name, bias in (("uniform", None), ("zipf", zipf)):
+            hs = [torch.randn((T, H), generator=gen, device=dev).to(torch.bfloat16) for _ in range(nbatch)]
+            y = torch.empty((T, H), dtype=torch.float32, device=dev)
+            touched = []
+            for i in range(nbatch):
+                _, ex = nv.moe_layer_decode(hs[i], wr, k, gu, dn, logit_bias=bias, y=y, want_routing=True, ws=wsd)
+                touched.append(int(torch.unique(ex["topk_idx"]).numel()))
+
+            def layer(i, bias=bias, hs=hs, y=y):
+                nv.moe_layer_decode(hs[i], wr, k, gu, dn, logit_bias=bias, y=y, ws=wsd)
+
+            torch.cuda.synchronize()
+            stream = torch.cuda.current_stream()
+            side = torch.cuda.Stream(device=dev)
+            side.wait_stream(stream)
+            graphs = []
+            with torch.cuda.stream(side):
+                for i in range(nbatch):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=side):
+                        layer(i)
+                    graphs.append(g)
+            stream.wait_stream(side)
+            t = _time_graphs(torch, graphs, max(reps, 2 * nbatch))
+            nbytes = sum(touched) / nbatch * MOE_EXPERT_BYTES + T * H * 6
+            out["runs"][f"T{T}_{bias_name}_fused"] = {"mode": "W4A16 fused layer (moe_layer_decode)",
+                                                     "us": round(t * 1e3, 2),
+                                                     "touched_experts_mean": round(sum(touched) / nbatch, 1),
+                                                     "GB/s": round(nbytes / (t * 1e-3) / 1e9, 1)}
     del gu, dn
     return out
 
@@ -628,7 +661,7 @@ def quantize_section(nv, torch, dev, reps=30):
 # ------------------------------------------------------------ profile cases ----
 
 CASES = ("decode_m1", "skinny_m4", "prefill_m2048", "quantize_m2048", "moe_t1", "moe_t32", "moe_t4096",
-         "stack_glue_m1")
+         "moe_fused_t1", "moe_fused_t32", "stack_glue_m1")
 
 
 def profile_case(args):
@@ -676,7 +709,7 @@ def profile_case(args):
             nv.nvfp4_quantize(x, sf_layout=nv.SF_TILED)
     else:
         E, H, I, k = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_K
-        T = int(case[len("moe_t"):])
+        T = int(case.rsplit("_t", 1)[1])
         mode = nv.MODE_W4A4 if T > 32 else nv.MODE_W4A16
 
         def stack(n, kk):
@@ -694,7 +727,12 @@ def profile_case(args):
         h = torch.randn((T, H), generator=gen, device=dev).to(torch.bfloat16)
         R = T * k
 
+        def run_fused():
+            nv.moe_layer_decode(h, wr, k, gu, dn)
+
         def run():
+            if case.startswith("moe_fused"):
+                return run_fused()
             r = nv.moe_route_topk(h, wr, k)
             a = nv.moe_grouped_linear(h, r["expert_offsets"], *gu, R, perm_tok=r["perm_tok"], gather=True,
                                       w_sf_layout=nv.SF_TILED, epilogue=nv.EPI_SWIGLU, y_dtype=torch.bfloat16,

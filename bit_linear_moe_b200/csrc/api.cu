@@ -349,10 +349,10 @@ struct MoeDecodeWs {
     float* topk_w;
     int32_t* n_groups;
     int32_t* groups;
-    int32_t* perm_t;
-    int32_t* perm_j;
-    int32_t* cnt;
+    void* h16;
     void* a;
+    void* a16;
+    float* inv_a;
     float* d;
     size_t bytes;
 };
@@ -366,11 +366,11 @@ static MoeDecodeWs moe_decode_ws(void* base, int64_t T, int64_t H, int64_t I, in
     w.topk_idx = (int32_t*)take(R * 4);
     w.topk_w = (float*)take(R * 4);
     w.n_groups = (int32_t*)take(16);
-    w.groups = (int32_t*)take(R * 12);
-    w.perm_t = (int32_t*)take(R * 4);
-    w.perm_j = (int32_t*)take(R * 4);
-    w.cnt = (int32_t*)take((size_t)(T * (H / 128)) * 4);
+    w.groups = (int32_t*)take(R * 32);
+    w.h16 = take((size_t)(T * H) * 2);
     w.a = take(R * (size_t)I * 2);
+    w.a16 = take(R * (size_t)I * 2);
+    w.inv_a = (float*)take(R * (size_t)(I / 64) * 4);
     w.d = (float*)take(R * (size_t)H * 4);
     w.bytes = off;
     return w;
@@ -378,7 +378,7 @@ static MoeDecodeWs moe_decode_ws(void* base, int64_t T, int64_t H, int64_t I, in
 
 static bool moe_decode_shape_ok(int64_t T, int64_t H, int64_t I, int32_t E, int32_t k) {
     return T >= 1 && T <= 32 && E >= 1 && E <= 1024 && k >= 1 && k <= 32 && k <= E && H >= 256 && H % 256 == 0 &&
-           I >= 256 && I % 256 == 0 && H <= 65536 && I <= 65536 && (int64_t)E * 2 * I < ((int64_t)1 << 31) &&
+           I >= 256 && I % 256 == 0 && H <= 4096 && I <= 4096 && (int64_t)E * 2 * I < ((int64_t)1 << 31) &&
            (int64_t)E * H < ((int64_t)1 << 31) && moe_decode_smem_bytes(H, I) <= 227 * 1024;
 }
 
@@ -425,10 +425,10 @@ int moe_layer_decode(const void* h, const void* w_router, const float* logit_bia
     L.topk_w = topk_w ? topk_w : w.topk_w;
     L.n_groups = w.n_groups;
     L.groups = w.groups;
-    L.perm_t = w.perm_t;
-    L.perm_j = w.perm_j;
-    L.cnt = w.cnt;
+    L.h16 = w.h16;
     L.a = a_out ? a_out : w.a;
+    L.a16 = w.a16;
+    L.inv_a = w.inv_a;
     L.d = w.d;
     L.y = y;
     L.y_dtype = y_dtype;

@@ -74,6 +74,11 @@ int launch_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales, const floa
                      int y_dtype, int* status, cudaStream_t st);
 
 // moe.cu
+// router_tc.cu: tensor-core router logits for T <= 64 (experts as M, split K
+// over a cluster; H % 64 == 0, 16-byte aligned rows), programmatic dependent
+bool router_tcs_supported(const void* h, const void* wr, int64_t T, int64_t H, int32_t E);
+int launch_router_logits_tcs(const void* h, const void* wr, const float* bias, int64_t T, int64_t H, int32_t E,
+                             float* logits, int* status, cudaStream_t st);
 // router_tc.cu: tensor-core router logits (T > 64, H % 64 == 0, 16-byte aligned rows)
 bool router_tc_supported(const void* h, const void* wr, int64_t T, int64_t H, int32_t E);
 int launch_router_logits_tc(const void* h, const void* wr, const float* bias, int64_t T, int64_t H, int32_t E,
@@ -106,7 +111,7 @@ int launch_gemm_w4a4_grouped(const uint8_t* a_codes, const uint8_t* a_scales, co
                              int y_dtype, int* status, cudaStream_t st);
 
 // moe_decode.cu: one routed expert layer for T <= 32 tokens (router, top-k,
-// gate/up + SwiGLU, down + combine), four kernels chained by PDL.
+// gate/up + SwiGLU, down, combine), five kernels chained by PDL.
 struct MoeDecodeLaunch {
     const void* h;              // [T, H] bf16
     const void* w_router;       // [E, H] bf16
@@ -122,11 +127,11 @@ struct MoeDecodeLaunch {
     int32_t* topk_idx;          // [T, k]
     float* topk_w;              // [T, k]
     int32_t* n_groups;          // routing tables: [1]
-    int32_t* groups;            // [T * k][3]
-    int32_t* perm_t;            // [T * k]
-    int32_t* perm_j;            // [T * k]
-    int32_t* cnt;               // [T][H / 128]
+    int32_t* groups;            // [T * k][8] token-group records
+    void* h16;                  // [T, H] fp16, h prescaled per token
     void* a;                    // [T * k, I] bf16
+    void* a16;                  // [T * k, I] fp16, a prescaled per (row, 64 columns)
+    float* inv_a;               // [T * k, I / 64]
     float* d;                   // [T * k, H]
     void* y;                    // [T, H]
     int y_dtype;

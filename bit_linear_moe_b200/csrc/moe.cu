@@ -145,6 +145,8 @@ int launch_router_logits_small_pdl(const void* h, const void* wr, const float* b
 
 int launch_router_logits(const void* h, const void* wr, const float* bias, int64_t T, int64_t H, int32_t E,
                          float* logits, cudaStream_t st) {
+    if (router_tcs_supported(h, wr, T, H, E))
+        return launch_router_logits_tcs(h, wr, bias, T, H, E, logits, device_status_ptr(), st);
     if (T <= 64 && H % 8 == 0) {
         const int64_t warps = (int64_t)E * ((T + kRouterTokGroup - 1) / kRouterTokGroup);
         router_logits_small_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(

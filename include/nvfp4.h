@@ -283,10 +283,10 @@ int moe_route_topk_noalloc(const void* h, const void* w_router, const float* log
  *   y          [T, H] in y_dtype (F32 or BF16)
  *   ws         scratch of moe_layer_decode_workspace(T, H, I, E, k) bytes;
  *              contents on entry are ignored.
- * The layer runs as four kernels chained by programmatic dependent launch.
- * Requires 1 <= T <= 32, 1 <= k <= 32, k <= E <= 1024, H % 256 == 0,
- * I % 256 == 0, TILED scales; the workspace query returns 0 for shapes out
- * of range. */
+ * The layer runs as five kernels chained by programmatic dependent launch.
+ * Requires 1 <= T <= 32, 1 <= k <= 32, k <= E <= 1024, H and I multiples of
+ * 256 and at most 4096, TILED scales; the workspace query returns 0 for
+ * shapes out of range. */
 size_t moe_layer_decode_workspace(int64_t T, int64_t H, int64_t I, int32_t E, int32_t k);
 int moe_layer_decode(const void* h, const void* w_router, const float* logit_bias,
                      int64_t T, int64_t H, int32_t E, int32_t k,

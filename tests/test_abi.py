@@ -244,3 +244,31 @@ def test_debug_wait_timeout_validation(L):
     assert L.nvfp4_debug_wait_timeout(5_000_000_000, None) == nv.ERR_SHAPE
     if not torch.cuda.is_available():
         assert L.nvfp4_debug_wait_timeout(1000, None) == nv.ERR_ARCH
+
+
+def test_moe_layer_decode_validation(L):
+    """The decode-time expert layer: workspace query and host-side checks."""
+    need = L.moe_layer_decode_workspace(32, 2048, 512, 512, 10)
+    assert need > 32 * 10 * 2048 * 4                      # holds the per-slot fp32 rows of the down projection
+    assert L.moe_layer_decode_workspace(33, 2048, 512, 512, 10) == 0    # T > 32
+    assert L.moe_layer_decode_workspace(1, 2000, 512, 512, 10) == 0     # H % 256
+    assert L.moe_layer_decode_workspace(1, 2048, 500, 512, 10) == 0     # I % 256
+    assert L.moe_layer_decode_workspace(1, 8192, 512, 512, 10) == 0     # H above 4096
+    assert L.moe_layer_decode_workspace(1, 2048, 512, 8, 10) == 0       # k > E
+
+    def call(**kw):
+        a = dict(h=FAKE, wr=FAKE, T=1, H=2048, E=512, k=10, I=512, y=FAKE2, yd=nv.DTYPE_F32, ws=FAKE2,
+                 wsb=L.moe_layer_decode_workspace(1, 2048, 512, 512, 10), ao=None)
+        a.update(kw)
+        return L.moe_layer_decode(a["h"], a["wr"], None, a["T"], a["H"], a["E"], a["k"], FAKE, FAKE, FAKE, a["I"],
+                                  FAKE, FAKE, FAKE, None, None, None, a["ao"], a["y"], a["yd"], a["ws"], a["wsb"],
+                                  None)
+
+    assert call(h=None) == nv.ERR_NULL
+    assert call(yd=5) == nv.ERR_DTYPE
+    assert call(T=0) == nv.ERR_SHAPE
+    assert call(T=40) == nv.ERR_SHAPE
+    assert call(ao=MISALIGNED) == nv.ERR_ALIGN
+    assert call(wsb=16) == nv.ERR_WORKSPACE
+    if not torch.cuda.is_available():
+        assert call() == nv.ERR_ARCH
