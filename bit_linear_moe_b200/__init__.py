@@ -28,6 +28,19 @@ MODE_AUTO, MODE_W4A16, MODE_W4A4 = 0, 1, 2
 EPI_NONE, EPI_SWIGLU, EPI_COMBINE = 0, 1, 2
 
 
+CHAIN_SRC_X, CHAIN_SRC_OP = 0, 1
+CHAIN_XFORM_NONE, CHAIN_XFORM_RMS, CHAIN_XFORM_SILU_MUL = 0, 1, 2
+
+
+class ChainOp(ctypes.Structure):
+    """``nvfp4_chain_op`` of include/nvfp4.h."""
+    _fields_ = [("w_codes", ctypes.c_void_p), ("w_scales", ctypes.c_void_p), ("w_gs", ctypes.c_void_p),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("src", ctypes.c_int32), ("src_op", ctypes.c_int32),
+                ("x", ctypes.c_void_p), ("x_ld", ctypes.c_int64), ("xform", ctypes.c_int32),
+                ("y_xform", ctypes.c_int32), ("y", ctypes.c_void_p), ("y_dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
 class NVFP4Error(RuntimeError):
     def __init__(self, status: int, call: str):
         super().__init__(f"{call} failed: {status_string(status)} (status {status})")
@@ -58,6 +71,8 @@ def lib() -> ctypes.CDLL:
             "nvfp4_linear": (i, [p, i, i64, i64, p, p, i, p, i64, p, i, i, p, sz, p]),
             "nvfp4_linear_w4a4q": (i, [p, p, p, i64, i64, p, p, p, i64, p, i, p]),
             "nvfp4_rms_norm": (i, [p, i, i64, i64, i64, p, p]),
+            "nvfp4_chain_workspace": (sz, [p, i32, i64]),
+            "nvfp4_chain": (i, [p, i32, i64, p, sz, p]),
             "nvfp4_silu_mul": (i, [p, i, i64, i64, p, p]),
             "moe_route_topk_workspace": (sz, [i64, i32, i32]),
             "moe_route_topk": (i, [p, p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p, sz, p]),
@@ -182,6 +197,44 @@ def nvfp4_linear_w4a4q(x_codes: torch.Tensor, x_scales: torch.Tensor, x_gs: torc
     _check(lib().nvfp4_linear_w4a4q(_ptr(x_codes), _ptr(x_scales), _ptr(x_gs), M, K, _ptr(w_codes), _ptr(w_scales),
                                     _ptr(w_gs), N, _ptr(y), _dtype_code(y), _stream()), "nvfp4_linear_w4a4q")
     return y
+
+
+def chain_ops(specs) -> "ctypes.Array":
+    """Build the ``nvfp4_chain_op`` array from dicts with keys ``w`` = (codes,
+    TILED scales, gs), ``src`` (a bf16 tensor [M, K] or the index of an earlier
+    op), ``K`` (when ``src`` is an op index: the columns the transform reads),
+    ``xform``, ``y`` (tensor or None) and ``y_xform``."""
+    arr = (ChainOp * len(specs))()
+    for i, sp in enumerate(specs):
+        c, sc, g = sp["w"]
+        o = arr[i]
+        o.w_codes, o.w_scales, o.w_gs = c.data_ptr(), sc.data_ptr(), g.data_ptr()
+        o.N, o.K = c.shape[0], c.shape[1] * 2
+        src = sp["src"]
+        if hasattr(src, "data_ptr"):
+            o.src, o.src_op, o.x, o.x_ld = CHAIN_SRC_X, -1, src.data_ptr(), src.stride(0)
+        else:
+            o.src, o.src_op, o.x, o.x_ld = CHAIN_SRC_OP, int(src), None, 0
+        o.xform = int(sp.get("xform", CHAIN_XFORM_NONE))
+        y = sp.get("y")
+        o.y = None if y is None else y.data_ptr()
+        o.y_dtype = DTYPE_F32 if y is None else _dtype_code(y)
+        o.y_xform = int(sp.get("y_xform", CHAIN_XFORM_NONE))
+    return arr
+
+
+def nvfp4_chain(specs, M: int, ws=None, ops=None):
+    """Run a list of W4A16 decode linears in one persistent launch per 12 ops
+    (see ``nvfp4_chain`` in include/nvfp4.h).  Outputs go to the ``y`` tensors
+    of the specs.  ``ops`` may pass a prebuilt :func:`chain_ops` array."""
+    if ops is None:
+        ops = chain_ops(specs)
+    n = len(ops)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    optr = ctypes.cast(ops, ctypes.c_void_p)
+    ws, wsb = _workspace(int(lib().nvfp4_chain_workspace(optr, n, M)), dev, ws)
+    _check(lib().nvfp4_chain(optr, n, M, _ptr(ws), wsb, _stream()), "nvfp4_chain")
+    return ws
 
 
 def moe_route_topk(h: torch.Tensor, w_router: torch.Tensor, k: int, logit_bias=None, want_logits: bool = False,

@@ -277,6 +277,21 @@ int nvfp4_linear_w4a4q(const uint8_t* x_codes, const uint8_t* x_scales, const fl
                             device_status_ptr(), (cudaStream_t)stream);
 }
 
+// ---- chains of decode linears ------------------------------------------------------
+
+size_t nvfp4_chain_workspace(const nvfp4_chain_op* ops, int32_t n_ops, int64_t M) {
+    return chain_workspace(ops, n_ops, M);
+}
+
+int nvfp4_chain(const nvfp4_chain_op* ops, int32_t n_ops, int64_t M, void* ws, size_t ws_bytes, void* stream) {
+    NVFP4_TRY(chain_validate(ops, n_ops, M));
+    const size_t need = chain_workspace(ops, n_ops, M);
+    if (!ws || ws_bytes < need) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NVFP4_ERR_ALIGN;
+    NVFP4_TRY(check_arch());
+    return launch_chain(ops, n_ops, M, ws, ws_bytes, device_status_ptr(), (cudaStream_t)stream);
+}
+
 // ---- decode-stack glue ---------------------------------------------------------------
 
 static bool float_dtype_ok(int d) { return d == NVFP4_DTYPE_F32 || d == NVFP4_DTYPE_BF16; }

@@ -92,6 +92,37 @@ NVFP4_DEV uint32_t f32x8_to_e2m1(const float (&v)[8]) {
     return out;
 }
 
+// ---- products ---------------------------------------------------------------
+
+// d = a * b + c with f16 a, b (exact product) and an fp32 accumulator.
+NVFP4_DEV float fma_f32_f16(uint16_t a, uint16_t b, float c) {
+    float d;
+    asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
+    return d;
+}
+
+// 32 products of one 16-byte chunk of E2M1 codes with 32 fp16 activations
+// (xw: 16 words of f16 pairs), as two 16-element block partials.  The f16
+// halves are taken as register halves (mov.b32 {lo, hi}), not by masking.
+NVFP4_DEV void dot32_e2m1_f16(const uint4& wq, const uint32_t* xw, float& p0, float& p1) {
+    const uint32_t w[4] = {wq.x, wq.y, wq.z, wq.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t h[4];
+        e2m1x8_to_f16x2(w[j], h);
+        float p = (j < 2) ? p0 : p1;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint16_t hl, hh, xl, xhi;
+            asm("mov.b32 {%0, %1}, %2;" : "=h"(hl), "=h"(hh) : "r"(h[q]));
+            asm("mov.b32 {%0, %1}, %2;" : "=h"(xl), "=h"(xhi) : "r"(xw[4 * j + q]));
+            p = fma_f32_f16(hl, xl, p);
+            p = fma_f32_f16(hh, xhi, p);
+        }
+        if (j < 2) p0 = p; else p1 = p;
+    }
+}
+
 // ---- scale layouts ----------------------------------------------------------
 
 // Byte offset of scale (r, c) of a matrix with `ncols_sf` scale columns.
@@ -103,6 +134,12 @@ NVFP4_DEV int64_t sf_offset(int64_t r, int64_t c, int64_t ncols_sf) {
         const int64_t cp4 = (ncols_sf + 3) >> 2;  // atoms along the scale columns
         return (((r >> 7) * cp4 + (c >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (c & 3);
     }
+}
+
+NVFP4_DEV float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
 }
 
 NVFP4_DEV float warp_sum(float v) {

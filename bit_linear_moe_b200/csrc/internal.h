@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/nvfp4.h"
+
 namespace nvfp4 {
 
 // Launch attribute for programmatic dependent launch (kernels that call
@@ -142,6 +144,12 @@ int launch_moe_decode(const MoeDecodeLaunch& L, cudaStream_t st);
 // the small-batch router kernel as a programmatic dependent launch
 int launch_router_logits_small_pdl(const void* h, const void* wr, const float* bias, int64_t T, int64_t H,
                                    int32_t E, float* logits, cudaStream_t st);
+
+// chain.cu: W4A16 decode linears in a persistent launch per 12 ops.
+int chain_validate(const nvfp4_chain_op* ops, int n_ops, int64_t M);
+size_t chain_workspace(const nvfp4_chain_op* ops, int n_ops, int64_t M);
+int launch_chain(const nvfp4_chain_op* ops, int n_ops, int64_t M, void* ws, size_t ws_bytes, int* status,
+                 cudaStream_t st);
 
 // Tokens per block of the routing permutation (top-k, counts, scatter): 32
 // gives one CTA per 32 tokens, so a 4,096-token batch spreads over 128 SMs.

@@ -281,29 +281,6 @@ __global__ void __launch_bounds__(1024) moe_decode_route_kernel(const float* __r
 
 // ---- expert projections ---------------------------------------------------------
 
-NVFP4_DEV float fma_f16hf(uint16_t a, uint16_t b, float c) {
-    float d;
-    asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(a), "h"(b), "f"(c));
-    return d;
-}
-
-// 32 code x activation products as two 16-element block partials.
-NVFP4_DEV void dot32h(const uint4& wq, const uint32_t* xw, float& p0, float& p1) {
-    const uint32_t w[4] = {wq.x, wq.y, wq.z, wq.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        uint32_t h[4];
-        e2m1x8_to_f16x2(w[j], h);
-        float p = (j < 2) ? p0 : p1;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint32_t xv = xw[4 * j + q];
-            p = fma_f16hf((uint16_t)(h[q] & 0xFFFF), (uint16_t)(xv & 0xFFFF), p);
-            p = fma_f16hf((uint16_t)(h[q] >> 16), (uint16_t)(xv >> 16), p);
-        }
-        if (j < 2) p0 = p; else p1 = p;
-    }
-}
 
 // PHASE 0: gate/up + SwiGLU (K = H, 64 + 64 rows per tile, I / 64 tiles per
 // group); PHASE 1: down (K = I, 128 rows per tile, H / 128 tiles per group).
@@ -495,7 +472,7 @@ __global__ void __launch_bounds__(moedec::kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         float p0 = 0.0f, p1 = 0.0f;
-                        dot32h(wq[i], xw, p0, p1);
+                        dot32_e2m1_f16(wq[i], xw, p0, p1);
                         acc[i][t] = fmaf(p0, sd[i].x * iv, acc[i][t]);
                         acc[i][t] = fmaf(p1, sd[i].y * iv, acc[i][t]);
                     }

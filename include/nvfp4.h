@@ -192,6 +192,52 @@ int nvfp4_linear_w4a4q(const uint8_t* x_codes, const uint8_t* x_scales, const fl
                        const uint8_t* w_codes, const uint8_t* w_scales, const float* w_gs, int64_t N,
                        void* y, int y_dtype, void* stream);
 
+/* ---- nvfp4_chain ----------------------------------------------------------
+ * A list of W4A16 decode linears run in order by one persistent launch (a
+ * launch per 12 ops): the decode chain of a layer stack, streamed without the
+ * drain, prologue and tail of a launch per linear (Ignis README, "The decode
+ * round": a decode step streams every layer's weights; "Credits": the decode
+ * chain replayed as one unit).
+ * Op i computes out_i = x_i W_i^T (W_i [N, K] NVFP4, TILED scales), M rows,
+ * with x_i taken from
+ *   SRC_X   a caller bf16 tensor x [M, K] (row stride x_ld elements), or
+ *   SRC_OP  the output v of an earlier op src_op of the same call, through
+ *           XFORM_NONE      x = bf16(v)                       (v has >= K columns)
+ *           XFORM_RMS       x = bf16(v[:, :K] / sqrt(mean(v[:, :K]^2)))
+ *                           (a row of zeros stays zero)
+ *           XFORM_SILU_MUL  x[:, j] = bf16(silu(v[:, j]) * v[:, K + j]),
+ *                           silu(a) = a / (1 + e^-a)        (v has 2K columns)
+ * and, if y is not NULL, writes y = out_i (XFORM_NONE) or y = rms(out_i)
+ * (XFORM_RMS, over all N columns) in y_dtype.  Ops without y keep their
+ * output in the workspace only.  Outputs accumulate in fp32 (the split-K
+ * partial sums of an output element are added in a fixed order: results are
+ * deterministic).
+ *   ws  scratch of nvfp4_chain_workspace(ops, n_ops, M) bytes; contents on
+ *       entry are ignored.
+ * Requires 1 <= M <= 2, K % 256 == 0, N % 8 == 0, 16-byte aligned pointers;
+ * needs two resident CTAs per SM (returns NVFP4_ERR_LAUNCH otherwise); a grid
+ * barrier that runs out reports NVFP4_ERR_DEVICE_TIMEOUT through
+ * nvfp4_read_device_status. */
+enum { NVFP4_CHAIN_SRC_X = 0, NVFP4_CHAIN_SRC_OP = 1 };
+enum { NVFP4_CHAIN_XFORM_NONE = 0, NVFP4_CHAIN_XFORM_RMS = 1, NVFP4_CHAIN_XFORM_SILU_MUL = 2 };
+typedef struct {
+    const uint8_t* w_codes;   /* [N, K/2] */
+    const uint8_t* w_scales;  /* TILED */
+    const float* w_gs;        /* [1] */
+    int64_t N, K;
+    int32_t src;              /* NVFP4_CHAIN_SRC_X or NVFP4_CHAIN_SRC_OP */
+    int32_t src_op;           /* SRC_OP: index of an earlier op */
+    const void* x;            /* SRC_X: bf16 [M, x_ld] */
+    int64_t x_ld;
+    int32_t xform;            /* SRC_OP: NVFP4_CHAIN_XFORM_*; SRC_X: NONE */
+    int32_t y_xform;          /* NONE or RMS */
+    void* y;                  /* NULL or [M, N] */
+    int32_t y_dtype;          /* F32 or BF16 */
+    int32_t reserved;
+} nvfp4_chain_op;
+size_t nvfp4_chain_workspace(const nvfp4_chain_op* ops, int32_t n_ops, int64_t M);
+int nvfp4_chain(const nvfp4_chain_op* ops, int32_t n_ops, int64_t M, void* ws, size_t ws_bytes, void* stream);
+
 /* ---- nvfp4_rms_norm / nvfp4_silu_mul -------------------------------------
  * The glue between the linears of a dense decode stack (Ignis README, "The
  * decode round": a decode step streams the whole stack's weights once).  The

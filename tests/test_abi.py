@@ -272,3 +272,41 @@ def test_moe_layer_decode_validation(L):
     assert call(wsb=16) == nv.ERR_WORKSPACE
     if not torch.cuda.is_available():
         assert call() == nv.ERR_ARCH
+
+
+def test_chain_validation(L):
+    import bit_linear_moe_b200 as nvm
+
+    class T:  # a stand-in tensor with a fixed aligned address
+        def __init__(self, ptr, shape, stride0=None, dtype=torch.float32):
+            self._p, self.shape, self.dtype = ptr, shape, dtype
+            self._s = stride0 if stride0 is not None else shape[-1]
+
+        def data_ptr(self):
+            return self._p
+
+        def stride(self, d):
+            return self._s
+
+    w = (T(0x10000, (128, 128)), T(0x20000, (128,)), T(0x30000, (1,)))
+    def run(specs, M=1):
+        ops = nvm.chain_ops(specs)
+        n = len(ops)
+        p = ctypes.cast(ops, ctypes.c_void_p)
+        need = L.nvfp4_chain_workspace(p, n, M)
+        return L.nvfp4_chain(p, n, M, FAKE2 if need else None, need, None), need
+
+    xin = T(0x40000, (1, 256), dtype=torch.bfloat16)
+    ok = [{"w": w, "src": xin, "y": T(0x50000, (1, 128))}]
+    st, need = run(ok)
+    assert need > 0
+    if not torch.cuda.is_available():
+        assert st == nv.ERR_ARCH
+    assert run(ok, M=3)[0] == nv.ERR_SHAPE                                         # M > 2
+    assert run([{"w": w, "src": 0}])[0] == nv.ERR_SHAPE                           # reads itself
+    assert run([{"w": w, "src": xin, "xform": nv.CHAIN_XFORM_RMS}])[0] == nv.ERR_MODE
+    assert run([{"w": w, "src": T(0x40008, (1, 256), dtype=torch.bfloat16)}])[0] == nv.ERR_ALIGN
+    w_bad = (T(0x10000, (100, 128)), w[1], w[2])                                    # N % 8
+    assert run([{"w": w_bad, "src": xin}])[0] == nv.ERR_SHAPE
+    two = ok + [{"w": w, "src": 0, "xform": nv.CHAIN_XFORM_SILU_MUL}]              # silu needs N = 2K
+    assert run(two)[0] == nv.ERR_SHAPE
