@@ -293,6 +293,7 @@ def run_native(args, rank, world, dist):
     extra = {"decode_m1_per_shape": per_shape}
     if not args.quick:
         extra["decode_sweep"] = decode_sweep(nv, torch, dev, layers)
+        extra["verify_widths"] = verify_section(nv, torch, dev, layers)
         extra["prefill"] = prefill_section(nv, torch, dev, layers)
         extra["quantize"] = quantize_section(nv, torch, dev)
         extra["moe_layer"] = moe_section(nv, torch, dev)
@@ -365,6 +366,35 @@ def decode_sweep(nv, torch, dev, layers, reps=20):
             del gr
         out[name] = row
         del many
+    return out
+
+
+def verify_section(nv, torch, dev, layers, reps=40):
+    """Speculative-verify widths (one target-model pass over 1 + draft tokens):
+    the decode step of the four linears at M in {8, 16, 64}, one CUDA graph
+    per width (and per weight copy), W4A16; for 64 tokens also AUTO, which
+    picks W4A4 above 32 tokens.  GB/s counts the step's algorithmic bytes."""
+    from bit_linear_moe_b200 import synth
+    out = {}
+    seeds = dict((s[0], s[3]) for s in SHAPES)
+    for M in synth.VERIFY_M:
+        modes = [("W4A16", nv.MODE_W4A16)] + ([("AUTO", nv.MODE_AUTO)] if M > 32 else [])
+        for mname, mode in modes:
+            xs = [torch.from_numpy(synth.decode_x(seeds[name], M, K)).to(torch.bfloat16).to(dev)
+                  for name, K, N, *_ in layers]
+            ys = [torch.empty((M, N), dtype=torch.float32, device=dev) for _, K, N, *_ in layers]
+            wss = [torch.empty(max(16, int(nv.lib().nvfp4_linear_workspace(M, K, N, mode))), dtype=torch.uint8,
+                               device=dev) for _, K, N, *_ in layers]
+
+            def step(i, xs=xs, ys=ys, wss=wss, mode=mode):
+                for j, (name, K, N, copies, _, _) in enumerate(layers):
+                    c, s_, g = copies[i % 2]
+                    nv.nvfp4_linear(xs[j], c, s_, g, w_sf_layout=nv.SF_TILED, y=ys[j], mode=mode, ws=wss[j])
+
+            t = _time_graphs(torch, _capture(torch, dev, step), reps)
+            nbytes = sum(decode_bytes(M, K, N) for _, K, N, *_ in layers)
+            out[f"M{M}_{mname}"] = {"us_per_step": round(t * 1e3, 2), "GB/s": round(nbytes / (t * 1e-3) / 1e9, 1),
+                                    "tokens_per_s_per_layer_step": round(M / (t * 1e-3), 1)}
     return out
 
 

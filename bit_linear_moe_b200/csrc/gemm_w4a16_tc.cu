@@ -46,7 +46,7 @@ namespace w4a16tc {
 constexpr int kStages = 3;
 constexpr int kCodes = 128 * 128, kSf = 2048;
 constexpr int kThreads = 320;
-constexpr int kTmemCols = 256;  // A ring: 6 x 32 columns, D: NT columns at 192
+constexpr int kTmemCols = 256;  // A ring: 6 x 32 columns, D: NT (<= 64) columns at 192
 constexpr int kAChunks = 6;
 template <int NT>
 struct Cfg {
@@ -69,11 +69,15 @@ struct TcArgs {
 
 template <int NT>
 NVFP4_DEV void tmem_ld_acc(uint32_t taddr, float (&v)[NT]) {
-    uint32_t r[32];
-    tmem_ld_32x32b_x32(taddr, r);  // reads 32 columns; columns >= NT are unused
-    tmem_ld_wait();
 #pragma unroll
-    for (int t = 0; t < NT; ++t) v[t] = __uint_as_float(r[t]);
+    for (int c0 = 0; c0 < NT; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + c0, r);  // 32 columns at a time; columns >= NT are unused
+        tmem_ld_wait();
+#pragma unroll
+        for (int t = 0; t < 32; ++t)
+            if (c0 + t < NT) v[c0 + t] = __uint_as_float(r[t]);
+    }
 }
 
 template <int NT, typename OutT>
@@ -280,11 +284,13 @@ static int run(TcArgs a, const uint8_t* codes, const void* xh, cudaStream_t st) 
     CUtensorMap mw, mx;
     if (!make_tmap_2d_u8(&mw, codes, (uint64_t)(a.K / 2), (uint64_t)a.N, 128, 128, 1)) return NVFP4_ERR_LAUNCH;
     if (!make_tmap_2d_u8(&mx, xh, (uint64_t)(a.K * 2), (uint64_t)a.M, 128, NT, 1)) return NVFP4_ERR_LAUNCH;
-    // split K so that there are about two CTAs per SM (two fit: ~80-104 KB of
-    // shared memory, 256 tensor-memory columns each)
+    // split K so that the grid is about one CTA per resident slot (two per SM
+    // for 16 and 32 tokens, ~80-104 KB of shared memory and 256 tensor-memory
+    // columns each; one per SM for 64 tokens, ~150 KB)
     const int64_t tiles = (a.N + 127) / 128;
     const int nst = (int)(a.K / 256);
-    int qs = (int)((2 * 148 + tiles / 2) / tiles);
+    const int slots = (Cfg<NT>::kSmemBytes <= 110 * 1024 ? 2 : 1) * 148;
+    int qs = (int)((slots + tiles / 2) / tiles);
     if (qs > 8) qs = 8;
     if (qs > nst) qs = nst;
     if (qs < 1) qs = 1;
@@ -305,7 +311,7 @@ static int run(TcArgs a, const uint8_t* codes, const void* xh, cudaStream_t st) 
 }
 
 bool w4a16_tc_supported(int64_t M, int64_t K, int64_t N, int sf_layout) {
-    return sf_layout == NVFP4_SF_TILED && M >= 3 && M <= 32 && K % 256 == 0 && N <= ((int64_t)1 << 30);
+    return sf_layout == NVFP4_SF_TILED && M >= 3 && M <= 64 && K % 256 == 0 && N <= ((int64_t)1 << 30);
 }
 
 int launch_w4a16_tc(const void* xh, const float* inv_scale, int64_t M, int64_t K, const uint8_t* codes,
@@ -325,8 +331,12 @@ int launch_w4a16_tc(const void* xh, const float* inv_scale, int64_t M, int64_t K
         if (y_dtype == NVFP4_DTYPE_BF16) return run<16, __nv_bfloat16>(a, codes, xh, st);
         return run<16, float>(a, codes, xh, st);
     }
-    if (y_dtype == NVFP4_DTYPE_BF16) return run<32, __nv_bfloat16>(a, codes, xh, st);
-    return run<32, float>(a, codes, xh, st);
+    if (M <= 32) {
+        if (y_dtype == NVFP4_DTYPE_BF16) return run<32, __nv_bfloat16>(a, codes, xh, st);
+        return run<32, float>(a, codes, xh, st);
+    }
+    if (y_dtype == NVFP4_DTYPE_BF16) return run<64, __nv_bfloat16>(a, codes, xh, st);
+    return run<64, float>(a, codes, xh, st);
 }
 
 }  // namespace nvfp4

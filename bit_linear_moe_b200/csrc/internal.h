@@ -58,7 +58,7 @@ int launch_x_prep(const void* x, const int32_t* gather, int64_t rows, int64_t K,
                   cudaStream_t st);
 int launch_gemv_w4a16(const GemvArgs& a, cudaStream_t st);
 
-// gemm_w4a16_tc.cu: W4A16 with dequantized weights in tensor memory (M <= 32, TILED, K % 256 == 0).
+// gemm_w4a16_tc.cu: W4A16 with dequantized weights in tensor memory (3 <= M <= 64, TILED, K % 256 == 0).
 bool w4a16_tc_supported(int64_t M, int64_t K, int64_t N, int sf_layout);
 int launch_w4a16_tc(const void* xh, const float* inv_scale, int64_t M, int64_t K, const uint8_t* codes,
                     const uint8_t* scales, const float* gs, int64_t N, void* y, int y_dtype, int* status,

@@ -34,6 +34,7 @@ DENSE27B = (
     ("down", 17408, 5120, 4),
 )
 DECODE_M = (1, 2, 4, 8, 16, 32)
+VERIFY_M = (8, 16, 64)          # speculative-verify widths: 1 + draft tokens
 PREFILL_M = (512, 2048, 8192)
 
 MOE_E, MOE_H, MOE_I, MOE_K = 512, 2048, 512, 10

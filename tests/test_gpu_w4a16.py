@@ -91,9 +91,10 @@ def test_degenerate_weights():
 
 
 @pytest.mark.parametrize("M,K,N", [(5, 256, 128), (8, 512, 200), (13, 1024, 1000), (16, 256, 64), (17, 768, 130),
-                                   (32, 5120, 256), (24, 2048, 384)])
+                                   (32, 5120, 256), (24, 2048, 384), (33, 256, 64), (48, 1024, 300),
+                                   (64, 5120, 256), (64, 768, 130)])
 def test_tensor_core_widths(M, K, N):
-    """Widths 5..32 with tensor-core scales run the tensor-memory kernel."""
+    """Widths 5..64 with tensor-core scales run the tensor-memory kernel."""
     rng = np.random.default_rng(M * 7 + K + N)
     q = oracle.quantize(synth.weight(rng, N, K))
     x = synth.activations(rng, M, K)
@@ -101,3 +102,15 @@ def test_tensor_core_widths(M, K, N):
     for y_dtype in (torch.float32, torch.bfloat16):
         y = _run(x, q, nv.SF_TILED, y_dtype)
         assert_within_bound(y, ref, ad, y_dtype == torch.bfloat16, f"tc {M}x{K}x{N}")
+
+
+@pytest.mark.parametrize("name,K,N,seed", synth.DENSE27B)
+def test_dense27b_verify_width_64(name, K, N, seed):
+    """The widest speculative-verify width (64 tokens) on the 27B-shaped
+    linears, W4A16, every output checked."""
+    M = 64
+    q = _dense_q(seed, K, N)
+    x = synth.decode_x(seed, M, K)
+    ref, ad = oracle.linear_w4a16(x, *q)
+    y = _run(x, q, nv.SF_TILED, torch.bfloat16)
+    assert_within_bound(y, ref, ad, True, f"{name} M={M}")
