@@ -72,6 +72,8 @@ def lib() -> ctypes.CDLL:
             "nvfp4_linear_w4a4q": (i, [p, p, p, i64, i64, p, p, p, i64, p, i, p]),
             "nvfp4_rms_norm": (i, [p, i, i64, i64, i64, p, p]),
             "nvfp4_chain_workspace": (sz, [p, i32, i64]),
+            "nvfp4_calibrate_workspace": (sz, [i64, i64, i64]),
+            "nvfp4_calibrate": (i, [p, i64, i64, p, i, i64, i, p, p, p, p, p, p, p, sz, p]),
             "nvfp4_chain": (i, [p, i32, i64, p, sz, p]),
             "nvfp4_silu_mul": (i, [p, i, i64, i64, p, p]),
             "moe_route_topk_workspace": (sz, [i64, i32, i32]),
@@ -146,6 +148,26 @@ def nvfp4_quantize(x: torch.Tensor, gs_in: torch.Tensor | None = None, sf_layout
     _check(lib().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, _ptr(gs_in), sf_layout, _ptr(codes),
                                 _ptr(scales), _ptr(gs_out), _ptr(ws), wsb, _stream()), "nvfp4_quantize")
     return codes, scales, gs_out
+
+
+def nvfp4_calibrate(w: torch.Tensor, x_calib: torch.Tensor, sf_layout: int = SF_ROWMAJOR, ws=None):
+    """Activation-calibrated quantization of ``w [N, K]`` (fp32) from ``x_calib
+    [S, K]`` (bf16).  Returns ``(codes, scales, gs, col_scale, err[9], alpha_idx)``:
+    the quantized ``w * col_scale``; use it on activations divided by ``col_scale``."""
+    N, K = w.shape
+    S = x_calib.shape[0]
+    dev = w.device
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(nvfp4_scales_bytes(N, K, sf_layout), dtype=torch.uint8, device=dev)
+    gs = torch.empty(1, dtype=torch.float32, device=dev)
+    col = torch.empty(K, dtype=torch.float32, device=dev)
+    err = torch.empty(9, dtype=torch.float32, device=dev)
+    aidx = torch.empty(1, dtype=torch.int32, device=dev)
+    ws, wsb = _workspace(int(lib().nvfp4_calibrate_workspace(N, K, S)), dev, ws)
+    _check(lib().nvfp4_calibrate(_ptr(w), N, K, _ptr(x_calib), _dtype_code(x_calib), S, sf_layout, _ptr(codes),
+                                 _ptr(scales), _ptr(gs), _ptr(col), _ptr(err), _ptr(aidx), _ptr(ws), wsb,
+                                 _stream()), "nvfp4_calibrate")
+    return codes, scales, gs, col, err, aidx
 
 
 def nvfp4_rms_norm(x: torch.Tensor, cols: int | None = None, y=None):

@@ -175,6 +175,54 @@ int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t cols, const
     return launch_quantize(x, x_dtype, nullptr, rows, cols, sf_layout, gs_in, amax, codes, scales, gs_out, st);
 }
 
+// ---- calibrated quantizer ----------------------------------------------------------
+
+static CalibrateWs calibrate_ws(void* base, int64_t N, int64_t K) {
+    CalibrateWs w{};
+    char* p = (char*)base;
+    size_t off = 0;
+    auto take = [&](size_t n) { char* q = p ? p + off : nullptr; off += align256(n); return q; };
+    w.a = (float*)take((size_t)K * 4);
+    w.m2 = (float*)take((size_t)K * 4);
+    w.s = (float*)take((size_t)K * 4 * 9);
+    w.w_scaled = (float*)take((size_t)(N * K) * 4);
+    w.amax = (unsigned*)take(16);
+    w.codes = (uint8_t*)take((size_t)(N * K / 2));
+    w.scales = (uint8_t*)take((size_t)(N * K / 16));
+    w.gs = (float*)take(16);
+    w.partial = (double*)take((size_t)kCalErrBlocks * 8);
+    w.err = (double*)take(9 * 8);
+    w.j_best = (int32_t*)take(16);
+    return w;
+}
+static size_t calibrate_ws_bytes(int64_t N, int64_t K) {
+    CalibrateWs w = calibrate_ws((void*)(uintptr_t)256, N, K);  // offsets from a stand-in base
+    return (size_t)((char*)w.j_best - (char*)(uintptr_t)256) + 256;
+}
+
+size_t nvfp4_calibrate_workspace(int64_t N, int64_t K, int64_t S) {
+    if (N < 1 || K < 16 || K % 16 || S < 1) return 0;
+    return calibrate_ws_bytes(N, K);
+}
+
+int nvfp4_calibrate(const float* w, int64_t N, int64_t K, const void* x, int x_dtype, int64_t S, int sf_layout,
+                    uint8_t* codes, uint8_t* scales, float* gs_out, float* col_scale_out, float* err_out,
+                    int32_t* alpha_idx_out, void* ws, size_t ws_bytes, void* stream) {
+    if (!w || !x || !codes || !scales || !gs_out || !col_scale_out) return NVFP4_ERR_NULL;
+    if (x_dtype != NVFP4_DTYPE_BF16) return NVFP4_ERR_DTYPE;
+    if (!layout_ok(sf_layout)) return NVFP4_ERR_LAYOUT;
+    if (N < 1 || K < 16 || K % 16 || S < 1 || N > ((int64_t)1 << 24) || K > ((int64_t)1 << 24) ||
+        N * K > ((int64_t)1 << 34) || S > ((int64_t)1 << 24))
+        return NVFP4_ERR_SHAPE;
+    if (!aligned16(w) || !aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(col_scale_out))
+        return NVFP4_ERR_ALIGN;
+    if (!ws || ws_bytes < calibrate_ws_bytes(N, K)) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NVFP4_ERR_ALIGN;
+    NVFP4_TRY(check_arch());
+    return launch_calibrate(w, N, K, x, S, sf_layout, codes, scales, gs_out, col_scale_out, err_out, alpha_idx_out,
+                            calibrate_ws(ws, N, K), (cudaStream_t)stream);
+}
+
 // ---- linear --------------------------------------------------------------------
 
 static int resolve_mode(int mode, int64_t M) {

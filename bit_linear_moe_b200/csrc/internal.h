@@ -151,6 +151,31 @@ size_t chain_workspace(const nvfp4_chain_op* ops, int n_ops, int64_t M);
 int launch_chain(const nvfp4_chain_op* ops, int n_ops, int64_t M, void* ws, size_t ws_bytes, int* status,
                  cudaStream_t st);
 
+// calibrate.cu: activation-calibrated quantization of a weight (9 alphas).
+constexpr int kCalErrBlocks = 296;
+struct CalibrateWs {
+    float* a;            // [K] mean |x|
+    float* m2;           // [K] mean x^2
+    float* s;            // [9][K] channel scales per alpha
+    float* w_scaled;     // [N, K]
+    unsigned* amax;
+    uint8_t* codes;      // [N, K/2]
+    uint8_t* scales;     // [N, K/16] row-major
+    float* gs;
+    double* partial;     // [kCalErrBlocks]
+    double* err;         // [9]
+    int32_t* j_best;
+};
+int launch_calibrate(const float* w, int64_t N, int64_t K, const void* x, int64_t S, int sf_layout, uint8_t* codes,
+                     uint8_t* scales, float* gs_out, float* col_scale_out, float* err_out, int32_t* alpha_idx_out,
+                     const CalibrateWs& ws, cudaStream_t st);
+
+#define NVFP4_TRY_INTERNAL(expr)        \
+    do {                                \
+        const int _s = (expr);          \
+        if (_s != NVFP4_OK) return _s;  \
+    } while (0)
+
 // Tokens per block of the routing permutation (top-k, counts, scatter): 32
 // gives one CTA per 32 tokens, so a 4,096-token batch spreads over 128 SMs.
 constexpr int kPermBlockTokens = 32;

@@ -143,6 +143,37 @@ int nvfp4_quantize(const void* x, int x_dtype, int64_t rows, int64_t cols,
                    uint8_t* codes, uint8_t* scales, float* gs_out,
                    void* ws, size_t ws_bytes, void* stream);
 
+/* ---- nvfp4_calibrate -------------------------------------------------------
+ * Activation-calibrated NVFP4 quantization of a weight (imp v0.20.0 release
+ * notes, "Highlights": a first-party NVFP4 quantizer with AWQ-class
+ * activation calibration).  From a calibration batch x [S, K] (bf16):
+ *     a_k  = (sum_s |x[s, k]|) / S,  m2_k = (sum_s x[s, k]^2) / S
+ *            (binary32, rows added in order)
+ *     for alpha = j / 8, j = 0..8:
+ *       s_k = a_k^alpha (1 where a_k == 0), then s_k /= sqrt(max s * min s);
+ *             a^(j/8) is computed from r1 = sqrt(a), r2 = sqrt(r1),
+ *             r3 = sqrt(r2) as 1, r3, r2, r2*r3, r1, r1*r3, r1*r2,
+ *             (r1*r2)*r3, a (IEEE square roots and products)
+ *       W'  = W diag(s) (binary32), quantized as nvfp4_quantize(W') (gs from
+ *             amax(W'))
+ *       err = sum_k m2_k sum_n (dequant(W')[n, k] / s_k - W[n, k])^2  (fp64)
+ *     the alpha of least err (lowest j on ties) is kept.
+ * The linear with the calibrated weight is y = (x / s) dequant(W')^T: the
+ * caller divides the activations by col_scale_out (or folds 1/s into the
+ * operation that produces them).  alpha = 0 is plain round-to-nearest.
+ *   w              [N, K] fp32 (device)
+ *   x              [S, K] bf16 calibration activations
+ *   codes, scales  out: W' in sf_layout;  gs_out one float
+ *   col_scale_out  out: s [K] of the chosen alpha
+ *   err_out        NULL or out [9]: err of every alpha (as float)
+ *   alpha_idx_out  NULL or out [1]: the chosen j (alpha = j / 8)
+ *   ws             scratch of nvfp4_calibrate_workspace(N, K, S) bytes.
+ * Requires K % 16 == 0. */
+size_t nvfp4_calibrate_workspace(int64_t N, int64_t K, int64_t S);
+int nvfp4_calibrate(const float* w, int64_t N, int64_t K, const void* x, int x_dtype, int64_t S, int sf_layout,
+                    uint8_t* codes, uint8_t* scales, float* gs_out, float* col_scale_out, float* err_out,
+                    int32_t* alpha_idx_out, void* ws, size_t ws_bytes, void* stream);
+
 /* ---- nvfp4_linear --------------------------------------------------------
  * y[m, n] = sum_k x[m, k] * W[n, k], W NVFP4 as above (Ignis README, "The
  * decode round"; imp home page, "How does it work?").

@@ -9,8 +9,9 @@ the seeded input generator module, which holds none of the method's arithmetic.
 The quantizer and the linears live in ``nvfp4_oracle.c`` (binary32 quantizer
 arithmetic in a fixed operation order, fp64 accumulation); the routing,
 permutation, SwiGLU and combine steps are plain numpy in :mod:`oracle.moe`,
-and the decode-stack glue (rms renormalisation, silu * up, bf16 rounding) in
-:mod:`oracle.stack`.
+the decode-stack glue (rms renormalisation, silu * up, bf16 rounding) in
+:mod:`oracle.stack`, and the activation-calibrated quantizer in
+:mod:`oracle.calibrate`.
 The format readings (rounding, ties, saturation, signed zero, zero-scale
 blocks, packing order) are stated in the C file's header.
 """

@@ -310,3 +310,23 @@ def test_chain_validation(L):
     assert run([{"w": w_bad, "src": xin}])[0] == nv.ERR_SHAPE
     two = ok + [{"w": w, "src": 0, "xform": nv.CHAIN_XFORM_SILU_MUL}]              # silu needs N = 2K
     assert run(two)[0] == nv.ERR_SHAPE
+
+
+def test_calibrate_validation(L):
+    def c(**kw):
+        a = dict(w=FAKE, N=64, K=128, x=FAKE2, xd=nv.DTYPE_BF16, S=16, lay=nv.SF_TILED)
+        a.update(kw)
+        need = L.nvfp4_calibrate_workspace(a["N"], a["K"], a["S"])
+        wsb = a.pop("wsb", need)
+        return L.nvfp4_calibrate(a["w"], a["N"], a["K"], a["x"], a["xd"], a["S"], a["lay"], FAKE, FAKE, FAKE, FAKE,
+                                 None, None, FAKE2 if wsb else None, wsb, None)
+    assert L.nvfp4_calibrate_workspace(64, 128, 16) > 64 * 128 * 4
+    assert L.nvfp4_calibrate_workspace(64, 100, 16) == 0
+    assert c(w=None) == nv.ERR_NULL
+    assert c(xd=nv.DTYPE_F32) == nv.ERR_DTYPE
+    assert c(K=100) == nv.ERR_SHAPE
+    assert c(S=0) == nv.ERR_SHAPE
+    assert c(lay=7) == nv.ERR_LAYOUT
+    assert c(wsb=64) == nv.ERR_WORKSPACE
+    if not torch.cuda.is_available():
+        assert c() == nv.ERR_ARCH
