@@ -294,7 +294,9 @@ def run_native(args, rank, world, dist):
     if not args.quick:
         extra["decode_sweep"] = decode_sweep(nv, torch, dev, layers)
         extra["verify_widths"] = verify_section(nv, torch, dev, layers)
-        extra["prefill"] = prefill_section(nv, torch, dev, layers)
+        extra["prefill"] = prefill_section(nv, torch, dev, layers, M=2048)
+        extra["prefill_m512"] = prefill_section(nv, torch, dev, layers, M=512)
+        extra["prefill_m8192"] = prefill_section(nv, torch, dev, layers, M=8192, reps=10)
         extra["quantize"] = quantize_section(nv, torch, dev)
         extra["moe_layer"] = moe_section(nv, torch, dev)
         try:
@@ -429,18 +431,31 @@ def _capture(torch, dev, fn_per_copy):
     return graphs
 
 
-def prefill_section(nv, torch, dev, layers, M=2048, reps=30):
-    """W4A4 prefill at M tokens on the four shapes: TFLOP/s = 2 M N K / time,
-    GEMM alone (pre-quantized activations) and with the activation quantize."""
+def prefill_section(nv, torch, dev, layers, M=2048, reps=30, library_ceiling=True):
+    """W4A4 prefill at M tokens on the four shapes: TFLOP/s = 2 M N K / time of
+      gemm        the GEMM alone (activations already NVFP4),
+      with_quant  nvfp4_linear(W4A4): amax pass + quantize pass + GEMM,
+      rms_*       a producer that renormalises the previous output first:
+                  unfused  nvfp4_rms_norm -> nvfp4_linear(W4A4)
+                  fused    nvfp4_rms_norm_quant -> nvfp4_linear_w4a4q,
+      library     torch's scaled_mm on the same NVFP4 operands (cuBLASLt, block
+                  scales 1x16 in the same swizzled layout): the measured FP4
+                  ceiling of this GPU."""
     from bit_linear_moe_b200 import synth
+    import torch.nn.functional as F
     seeds = dict((s[0], s[3]) for s in SHAPES)
     out = {"M": M, "shapes": {}}
-    tot_flop = tot_gemm = tot_e2e = 0.0
+    tot = {"flop": 0.0, "gemm": 0.0, "with_quant": 0.0, "rms_unfused": 0.0, "rms_fused": 0.0, "library": 0.0}
     for name, K, N, copies, _, _ in layers:
         x = torch.from_numpy(synth.prefill_x(seeds[name], M, K)[0]).to(torch.bfloat16).to(dev)
         xc, xs, xg = nv.nvfp4_quantize(x, sf_layout=nv.SF_TILED)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         ws = torch.empty(int(nv.lib().nvfp4_linear_workspace(M, K, N, nv.MODE_W4A4)), dtype=torch.uint8, device=dev)
+        xr = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        rq_ws = torch.empty(max(16, int(nv.lib().nvfp4_rms_norm_quant_workspace(M))), dtype=torch.uint8, device=dev)
+        rc = torch.empty_like(xc)
+        rs = torch.empty_like(xs)
+        rg = torch.empty_like(xg)
 
         def gemm(i):
             c, s, g = copies[i]
@@ -450,19 +465,53 @@ def prefill_section(nv, torch, dev, layers, M=2048, reps=30):
             c, s, g = copies[i]
             nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A4, ws=ws)
 
-        t_g = _time_graphs(torch, _capture(torch, dev, gemm), reps)
-        t_e = _time_graphs(torch, _capture(torch, dev, e2e), reps)
+        def rms_unfused(i):
+            c, s, g = copies[i]
+            nv.nvfp4_rms_norm(x, y=xr)
+            nv.nvfp4_linear(xr, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A4, ws=ws)
+
+        def rms_fused(i):
+            c, s, g = copies[i]
+            lib = nv.lib()
+            nv._check(lib.nvfp4_rms_norm_quant(nv._ptr(x), nv.DTYPE_BF16, M, K, K, nv.SF_TILED, nv._ptr(rc),
+                                               nv._ptr(rs), nv._ptr(rg), nv._ptr(rq_ws), rq_ws.numel(), nv._stream()),
+                      "nvfp4_rms_norm_quant")
+            nv.nvfp4_linear_w4a4q(rc, rs, rg, c, s, g, y=y)
+
         flop = 2.0 * M * N * K
-        out["shapes"][name] = {"gemm_us": round(t_g * 1e3, 1), "gemm_TFLOPs": round(flop / (t_g * 1e-3) / 1e12, 1),
-                               "with_quant_us": round(t_e * 1e3, 1),
-                               "with_quant_TFLOPs": round(flop / (t_e * 1e-3) / 1e12, 1)}
-        tot_flop += flop
-        tot_gemm += t_g
-        tot_e2e += t_e
-    out["gemm_TFLOPs"] = round(tot_flop / (tot_gemm * 1e-3) / 1e12, 1)
-    out["with_quant_TFLOPs"] = round(tot_flop / (tot_e2e * 1e-3) / 1e12, 1)
+        row = {}
+        for key, fn in (("gemm", gemm), ("with_quant", e2e), ("rms_unfused", rms_unfused), ("rms_fused", rms_fused)):
+            t = _time_graphs(torch, _capture(torch, dev, fn), reps)
+            row[key + "_us"] = round(t * 1e3, 1)
+            row[key + "_TFLOPs"] = round(flop / (t * 1e-3) / 1e12, 1)
+            tot[key] += t
+        if library_ceiling:
+            try:
+                a4, sa = xc.view(torch.float4_e2m1fn_x2), xs.view(torch.float8_e4m3fn)
+
+                def lib_mm(i):
+                    c, s, g = copies[i]
+                    F.scaled_mm(a4, c.view(torch.float4_e2m1fn_x2).t(), [sa], [F.ScalingType.BlockWise1x16],
+                                [s.view(torch.float8_e4m3fn)], [F.ScalingType.BlockWise1x16],
+                                swizzle_a=[F.SwizzleType.SWIZZLE_32_4_4], swizzle_b=[F.SwizzleType.SWIZZLE_32_4_4],
+                                output_dtype=torch.bfloat16)
+
+                t = _time_graphs(torch, _capture(torch, dev, lib_mm), reps)
+                row["library_us"] = round(t * 1e3, 1)
+                row["library_TFLOPs"] = round(flop / (t * 1e-3) / 1e12, 1)
+                tot["library"] += t
+            except Exception as exc:  # reported, not fatal: the ceiling is context
+                row["library"] = f"unavailable: {type(exc).__name__}: {str(exc)[:120]}"
+                tot["library"] = float("nan")
+        out["shapes"][name] = row
+        tot["flop"] += flop
+    for key in ("gemm", "with_quant", "rms_unfused", "rms_fused", "library"):
+        if tot[key] == tot[key] and tot[key] > 0:
+            out[key + "_TFLOPs"] = round(tot["flop"] / (tot[key] * 1e-3) / 1e12, 1)
     out["peak_nominal_dense_nvfp4_TFLOPs"] = 9000.0
     out["frac_of_nominal"] = round(out["gemm_TFLOPs"] / 9000.0, 4)
+    if out.get("library_TFLOPs"):
+        out["frac_of_library"] = round(out["gemm_TFLOPs"] / out["library_TFLOPs"], 4)
     return out
 
 

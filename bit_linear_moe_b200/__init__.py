@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             "nvfp4_calibrate": (i, [p, i64, i64, p, i, i64, i, p, p, p, p, p, p, p, sz, p]),
             "nvfp4_chain": (i, [p, i32, i64, p, sz, p]),
             "nvfp4_silu_mul": (i, [p, i, i64, i64, p, p]),
+            "nvfp4_rms_norm_quant_workspace": (sz, [i64]),
+            "nvfp4_rms_norm_quant": (i, [p, i, i64, i64, i64, i, p, p, p, p, sz, p]),
             "moe_route_topk_workspace": (sz, [i64, i32, i32]),
             "moe_route_topk": (i, [p, p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p, sz, p]),
             "moe_route_topk_noalloc": (i, [p, p, p, i64, i64, i32, i32, p, p, p, p, p, p, p, p]),
@@ -181,6 +183,22 @@ def nvfp4_rms_norm(x: torch.Tensor, cols: int | None = None, y=None):
         y = torch.empty((rows, cols), dtype=torch.bfloat16, device=x.device)
     _check(lib().nvfp4_rms_norm(_ptr(x), _dtype_code(x), rows, cols, ld, _ptr(y), _stream()), "nvfp4_rms_norm")
     return y
+
+
+def nvfp4_rms_norm_quant(x: torch.Tensor, cols: int | None = None, sf_layout: int = SF_TILED, ws=None):
+    """NVFP4 ``(codes, scales, gs)`` of ``nvfp4_rms_norm(x, cols)``, without the bf16 rows."""
+    rows, ld = x.shape
+    if x.stride(1) != 1 or x.stride(0) != ld:
+        raise ValueError("x must be a contiguous [rows, ld] tensor")
+    cols = ld if cols is None else int(cols)
+    dev = x.device
+    codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(nvfp4_scales_bytes(rows, cols, sf_layout), dtype=torch.uint8, device=dev)
+    gs = torch.empty(1, dtype=torch.float32, device=dev)
+    ws, wsb = _workspace(int(lib().nvfp4_rms_norm_quant_workspace(rows)), dev, ws)
+    _check(lib().nvfp4_rms_norm_quant(_ptr(x), _dtype_code(x), rows, cols, ld, sf_layout, _ptr(codes), _ptr(scales),
+                                      _ptr(gs), _ptr(ws), wsb, _stream()), "nvfp4_rms_norm_quant")
+    return codes, scales, gs
 
 
 def nvfp4_silu_mul(g: torch.Tensor, h=None):

@@ -358,6 +358,32 @@ int nvfp4_rms_norm(const void* x, int x_dtype, int64_t rows, int64_t cols, int64
     return launch_rms_norm(x, x_dtype, rows, cols, ld, y, (cudaStream_t)stream);
 }
 
+size_t nvfp4_rms_norm_quant_workspace(int64_t rows) {
+    if (rows < 1) return 0;
+    return align256(16) + align256((size_t)rows * 4);
+}
+
+int nvfp4_rms_norm_quant(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld, int sf_layout,
+                         uint8_t* codes, uint8_t* scales, float* gs_out, void* ws, size_t ws_bytes, void* stream) {
+    if (!x || !codes || !scales || !gs_out) return NVFP4_ERR_NULL;
+    if (!float_dtype_ok(x_dtype)) return NVFP4_ERR_DTYPE;
+    if (!layout_ok(sf_layout)) return NVFP4_ERR_LAYOUT;
+    if (rows < 1 || cols < 16 || cols % 16 || ld < cols || rows > ((int64_t)1 << 31) - 1 ||
+        cols > ((int64_t)1 << 31) || ld > ((int64_t)1 << 40) / rows)
+        return NVFP4_ERR_SHAPE;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || ld % (x_dtype == NVFP4_DTYPE_F32 ? 4 : 8))
+        return NVFP4_ERR_ALIGN;
+    if (!ws || ws_bytes < nvfp4_rms_norm_quant_workspace(rows)) return NVFP4_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NVFP4_ERR_ALIGN;
+    NVFP4_TRY(check_arch());
+    cudaStream_t st = (cudaStream_t)stream;
+    unsigned* amax = (unsigned*)ws;
+    float* inv = (float*)((char*)ws + align256(16));
+    NVFP4_TRY(launch_rms_stats(x, x_dtype, rows, cols, ld, inv, amax, st));
+    return launch_quantize(x, x_dtype, nullptr, rows, cols, sf_layout, nullptr, amax, codes, scales, gs_out, st,
+                           nullptr, ld, inv);
+}
+
 int nvfp4_silu_mul(const void* g, int g_dtype, int64_t rows, int64_t half, void* h, void* stream) {
     if (!g || !h) return NVFP4_ERR_NULL;
     if (!float_dtype_ok(g_dtype)) return NVFP4_ERR_DTYPE;

@@ -19,14 +19,22 @@ inline void set_pdl_attr(cudaLaunchAttribute& a) {
 // stack.cu: decode-stack glue (bf16 outputs)
 int launch_rms_norm(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld, void* y, cudaStream_t st);
 int launch_silu_mul(const void* g, int g_dtype, int64_t rows, int64_t half, void* h, cudaStream_t st);
+// The rms factor of every row (written to inv) and the largest |bf16(x * inv)|
+// over all rows (atomicMax into *amax_bits, zeroed first): the same reduction
+// as launch_rms_norm, so bf16(x * inv) equals its output.
+int launch_rms_stats(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld, float* inv,
+                     unsigned* amax_bits, cudaStream_t st);
 
 // quantize.cu
 int launch_amax(const void* x, int x_dtype, int64_t n, unsigned* amax_bits, cudaStream_t st);
 // src_rows (nullable): dst row r quantizes source row src_rows[r]; -1 = zero row.
 // row_bound (nullable, device): rows >= *row_bound are skipped entirely.
+// x_ld (0: cols) is the source row stride; row_inv (nullable, device): source
+// row r is normalised first, x -> bf16(x * row_inv[r]).
 int launch_quantize(const void* x, int x_dtype, const int32_t* src_rows, int64_t dst_rows, int64_t cols,
                     int sf_layout, const float* gs_in, const unsigned* amax_bits, uint8_t* codes,
-                    uint8_t* scales, float* gs_out, cudaStream_t st, const int32_t* row_bound = nullptr);
+                    uint8_t* scales, float* gs_out, cudaStream_t st, const int32_t* row_bound = nullptr,
+                    int64_t x_ld = 0, const float* row_inv = nullptr);
 // amax over bf16 rows x[src_rows[r]], r < nrows (negative entries skipped).
 int launch_amax_rows(const void* x, const int32_t* src_rows, int64_t nrows, int64_t cols, unsigned* amax_bits,
                      cudaStream_t st);

@@ -106,12 +106,16 @@ NVFP4_DEV float global_scale_from(const float* gs_in, const unsigned* amax_bits)
 // src_rows (nullable): dst row r reads source row src_rows[r]; -1 marks a
 // padding row (zero codes and scales).  Rows >= dst_rows (tiled padding) and
 // scale columns >= cols/16 get zero scales and no codes.
+// row_inv (nullable): source row r is first normalised, x -> bf16(x * row_inv[r])
+// (the rows of nvfp4_rms_norm, recomputed instead of read back); x_ld is the
+// source row stride in elements.
 template <typename T, int LAYOUT>
 __global__ void __launch_bounds__(256) quantize_kernel(
     const T* __restrict__ x, const int32_t* __restrict__ src_rows, int64_t dst_rows, int64_t cols,
     int64_t grid_rows, int64_t grid_cols, const float* __restrict__ gs_in,
     const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-    float* __restrict__ gs_out, const int32_t* __restrict__ row_bound) {
+    float* __restrict__ gs_out, const int32_t* __restrict__ row_bound, int64_t x_ld,
+    const float* __restrict__ row_inv) {
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     const float gs = global_scale_from(gs_in, amax_bits);
     if (i == 0 && gs_out) *gs_out = gs;
@@ -128,7 +132,12 @@ __global__ void __launch_bounds__(256) quantize_kernel(
         return;
     }
     float v[16];
-    Vec16<T>::load(x + src * cols + b * 16, v);
+    Vec16<T>::load(x + src * x_ld + b * 16, v);
+    if (row_inv) {
+        const float inv = row_inv[src];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = __bfloat162float(__float2bfloat16_rn(v[j] * inv));
+    }
     float amax_b = 0.0f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) amax_b = fmaxf(amax_b, fabsf(v[j]));
@@ -179,14 +188,17 @@ int launch_amax_rows(const void* x, const int32_t* src_rows, int64_t nrows, int6
 
 int launch_quantize(const void* x, int x_dtype, const int32_t* src_rows, int64_t dst_rows, int64_t cols,
                     int sf_layout, const float* gs_in, const unsigned* amax_bits, uint8_t* codes,
-                    uint8_t* scales, float* gs_out, cudaStream_t st, const int32_t* row_bound) {
+                    uint8_t* scales, float* gs_out, cudaStream_t st, const int32_t* row_bound, int64_t x_ld,
+                    const float* row_inv) {
+    if (x_ld <= 0) x_ld = cols;
     const int64_t nsf = cols / 16;
     const int64_t grid_rows = sf_layout == NVFP4_SF_TILED ? (dst_rows + 127) / 128 * 128 : dst_rows;
     const int64_t grid_cols = sf_layout == NVFP4_SF_TILED ? (nsf + 3) / 4 * 4 : nsf;
     const int grid = grid_for(grid_rows * grid_cols, 256);
 #define NVFP4_Q(T, L)                                                                                 \
     quantize_kernel<T, L><<<grid, 256, 0, st>>>((const T*)x, src_rows, dst_rows, cols, grid_rows,     \
-                                                grid_cols, gs_in, amax_bits, codes, scales, gs_out, row_bound)
+                                                grid_cols, gs_in, amax_bits, codes, scales, gs_out, row_bound, \
+                                                x_ld, row_inv)
     if (x_dtype == NVFP4_DTYPE_BF16) {
         if (sf_layout == NVFP4_SF_TILED) NVFP4_Q(__nv_bfloat16, NVFP4_SF_TILED);
         else NVFP4_Q(__nv_bfloat16, NVFP4_SF_ROWMAJOR);

@@ -286,6 +286,23 @@ int nvfp4_chain(const nvfp4_chain_op* ops, int32_t n_ops, int64_t M, void* ws, s
  *   g      [rows, 2 * half], g_dtype F32 or BF16;  h  [rows, half] bf16
  * Element-size alignment only; no workspace. */
 int nvfp4_rms_norm(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld, void* y, void* stream);
+
+/* nvfp4_rms_norm_quant:  the NVFP4 quantization of nvfp4_rms_norm(x) without
+ * writing or reading back its bf16 rows (Ignis README, "Credits": activations
+ * reach the prefill GEMM as NVFP4; the rms renormalisation is the producer).
+ * codes, scales and gs_out equal, bit for bit, nvfp4_quantize of the rows
+ * nvfp4_rms_norm(x, ...) returns, with gs_in = NULL: one pass takes each row's
+ * rms factor and the largest normalised magnitude over all rows (the global
+ * scale), a second writes codes and scales from x directly.  Feed the result
+ * to nvfp4_linear_w4a4q (sf_layout TILED).
+ *   x       rows of `cols` elements at stride ld (F32 or BF16), 16-byte
+ *           aligned, ld a multiple of 8 (BF16) or 4 (F32)
+ *   codes   out [rows, cols/2];  scales  out in sf_layout;  gs_out  out [1]
+ *   ws      scratch of nvfp4_rms_norm_quant_workspace(rows) bytes.
+ * Requires cols % 16 == 0. */
+size_t nvfp4_rms_norm_quant_workspace(int64_t rows);
+int nvfp4_rms_norm_quant(const void* x, int x_dtype, int64_t rows, int64_t cols, int64_t ld, int sf_layout,
+                         uint8_t* codes, uint8_t* scales, float* gs_out, void* ws, size_t ws_bytes, void* stream);
 int nvfp4_silu_mul(const void* g, int g_dtype, int64_t rows, int64_t half, void* h, void* stream);
 
 /* ---- moe_route_topk ------------------------------------------------------

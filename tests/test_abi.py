@@ -330,3 +330,20 @@ def test_calibrate_validation(L):
     assert c(wsb=64) == nv.ERR_WORKSPACE
     if not torch.cuda.is_available():
         assert c() == nv.ERR_ARCH
+
+
+def test_rms_norm_quant_validation(L):
+    def r(**kw):
+        a = dict(x=FAKE, xd=nv.DTYPE_BF16, rows=4, cols=64, ld=64, lay=nv.SF_TILED)
+        a.update(kw)
+        wsb = a.pop("wsb", L.nvfp4_rms_norm_quant_workspace(a["rows"]))
+        return L.nvfp4_rms_norm_quant(a["x"], a["xd"], a["rows"], a["cols"], a["ld"], a["lay"], FAKE, FAKE, FAKE2,
+                                      FAKE2, wsb, None)
+    assert r(x=None) == nv.ERR_NULL
+    assert r(xd=5) == nv.ERR_DTYPE
+    assert r(cols=40) == nv.ERR_SHAPE
+    assert r(ld=60) == nv.ERR_SHAPE
+    assert r(ld=68) == nv.ERR_ALIGN                      # bf16 rows need a stride of 8 elements
+    assert r(wsb=4) == nv.ERR_WORKSPACE
+    if not torch.cuda.is_available():
+        assert r() == nv.ERR_ARCH
