@@ -50,6 +50,16 @@ def decode_bytes(M, K, N):
     return N * K // 2 + N * K // 16 + M * K * 2 + 4
 
 
+STEP_BYTES = sum(decode_bytes(1, K, N) for _, K, N, _ in SHAPES)
+
+
+def workload_config(world: int) -> dict:
+    """The headline workload, identical in both arms' lines."""
+    return {"workload": WORKLOAD, "M": 1, "bytes_per_step": STEP_BYTES,
+            "l2": "weights 194.7 MB per step > 126 MB L2 (the native arm rotates 2 copies, 389 MB)",
+            "parallelism": f"replicas x{world}"}
+
+
 def max_over_ranks(ms: float, dist, device) -> float:
     """The slowest rank's time (every rank gets it); ``ms`` unchanged on one rank."""
     if not dist:
@@ -261,20 +271,39 @@ def run_native(args, rank, world, dist):
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
     traffic = kernel_traffic("gemv_tma.cu", "gemv_tma_decode")
 
-    # end to end through the public API: pinned host x in, host y out, every step
-    xh = [torch.empty((1, K), dtype=torch.bfloat16).pin_memory() for _, K, *_ in layers]
-    for h_, (_, K, N, c, x, y) in zip(xh, layers):
-        h_.copy_(x.cpu())
-    yh = [torch.empty((1, N), dtype=torch.float32).pin_memory() for _, K, N, *_ in layers]
-    h2d = sum(t.numel() * t.element_size() for t in xh)
-    d2h = sum(t.numel() * t.element_size() for t in yh)
+    # end to end through the C ABI: every step copies the four inputs from one
+    # pinned host buffer, calls nvfp4_linear four times (arguments marshalled
+    # once, as a C caller holds them) and copies the four outputs back to one
+    # pinned host buffer
+    import ctypes
+    ks, ns = [K for _, K, *_ in layers], [N for _, K, N, *_ in layers]
+    xh = torch.empty(sum(ks), dtype=torch.bfloat16).pin_memory()
+    xh.copy_(torch.cat([x.reshape(-1).cpu() for *_, x, y in layers]))
+    yh = torch.empty(sum(ns), dtype=torch.float32).pin_memory()
+    xd = torch.empty(sum(ks), dtype=torch.bfloat16, device=dev)
+    yd = torch.empty(sum(ns), dtype=torch.float32, device=dev)
+    h2d, d2h = xh.numel() * xh.element_size(), yh.numel() * yh.element_size()
+    cstream = ctypes.c_void_p(stream.cuda_stream)
+    abi_args = [[], []]
+    xo, yo = 0, 0
+    for (name, K, N, copies, x, y) in layers:
+        wsp = ws[name]
+        for i in range(2):
+            c, s_, g_ = copies[i]
+            abi_args[i].append((ctypes.c_void_p(xd[xo:].data_ptr()), nv.DTYPE_BF16, 1, K, ctypes.c_void_p(c.data_ptr()),
+                                ctypes.c_void_p(s_.data_ptr()), nv.SF_TILED, ctypes.c_void_p(g_.data_ptr()), N,
+                                ctypes.c_void_p(yd[yo:].data_ptr()), nv.DTYPE_F32, nv.MODE_W4A16,
+                                None if wsp is None else ctypes.c_void_p(wsp.data_ptr()),
+                                0 if wsp is None else wsp.numel(), cstream))
+        xo, yo = xo + K, yo + N
+    linear = nv.lib().nvfp4_linear
 
     def e2e_step(i):
-        for j, (name, K, N, copies, x, y) in enumerate(layers):
-            c, s, g = copies[i % 2]
-            x.copy_(xh[j], non_blocking=True)
-            nv.nvfp4_linear(x, c, s, g, w_sf_layout=nv.SF_TILED, y=y, mode=nv.MODE_W4A16, ws=ws[name])
-            yh[j].copy_(y, non_blocking=True)
+        xd.copy_(xh, non_blocking=True)
+        for a in abi_args[i % 2]:
+            if linear(*a) != 0:
+                raise RuntimeError("nvfp4_linear failed in the end-to-end step")
+        yh.copy_(yd, non_blocking=True)
 
     for i in range(args.warmup):
         e2e_step(i)
@@ -309,10 +338,8 @@ def run_native(args, rank, world, dist):
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 weights x bf16 activations, fp32 accumulate",
         "data": "synthetic: weights N(0,0.02) fp32 quantized on device, activations N(0,1) bf16",
-        "config": {"workload": WORKLOAD, "M": 1, "bytes_per_step": step_bytes,
-                   "timing": "CUDA-graph replay of the step (4 linears), events on the launching stream",
-                   "l2": "weights rotated over 2 copies (389 MB) > 126 MB L2",
-                   "parallelism": f"replicas x{world}"},
+        "config": workload_config(world),
+        "timing": "CUDA-graph replay of the step (4 linears), events on the launching stream",
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
                      "per": "decode step (4 launches, one per shape): algorithmic bytes / step time on this GPU",
@@ -828,59 +855,182 @@ def profile_case(args):
 
 # --------------------------------------------------------------- reference ----
 
+_ORACLE_W = {}
+
+
+def oracle_weights(row_frac: int = 1):
+    """The four linears' weights quantized by the oracle (every row_frac-th
+    row), with their M = 1 inputs: [(K, N, (codes, scales, gs), x)]."""
+    import oracle
+    from bit_linear_moe_b200 import synth
+    if row_frac not in _ORACLE_W:
+        qs = []
+        for name, K, N, seed in SHAPES:
+            c, s_, g = oracle.quantize(synth.dense_weight(seed, K, N)[::row_frac])
+            qs.append((K, c.shape[0], (c, s_, g), synth.decode_x(seed, 1, K)))
+        _ORACLE_W[row_frac] = qs
+    return _ORACLE_W[row_frac]
+
+
+def _rate(fn, units: float, seconds: float):
+    """(units per second, seconds, passes) of fn repeated for at least ``seconds``."""
+    t = time.perf_counter()
+    n = 0
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t
+        if dt >= seconds:
+            return units * n / dt, dt, n
+
+
 def oracle_decode_sample(min_seconds: float = 10.0, row_frac: int = 1):
     """Time the oracle's W4A16 linear on the same four shapes at M = 1 (weights
     quantized by the oracle outside the timed region), repeating the four
     linears until ``min_seconds`` have passed.  ``row_frac`` > 1 keeps every
     row_frac-th weight row (a bounded sample).  Returns (GB/s, seconds, passes, threads)."""
     import oracle
-    from bit_linear_moe_b200 import synth
-    qs = []
-    for name, K, N, seed in SHAPES:
-        c, s_, g = oracle.quantize(synth.dense_weight(seed, K, N)[::row_frac])
-        qs.append((K, c.shape[0], (c, s_, g), synth.decode_x(seed, 1, K)))
-    t = time.perf_counter()
-    nbytes, passes = 0, 0
-    while True:
-        for K, N, q, x in qs:
-            oracle.linear_w4a16(x, *q)
-            nbytes += decode_bytes(1, K, N)
-        passes += 1
-        dt = time.perf_counter() - t
-        if dt >= min_seconds:
-            break
-    return nbytes / dt / 1e9, dt, passes, oracle.num_threads()
-
-
-def run_reference(args):
-    """The oracle as the reference arm: each step is the four linears at M = 1
-    over every 64th weight row (a bounded sample of the workload)."""
-    import oracle
-    from bit_linear_moe_b200 import synth
-    qs = []
-    for name, K, N, seed in SHAPES:
-        c, s_, g = oracle.quantize(synth.dense_weight(seed, K, N)[::64])
-        qs.append((K, c.shape[0], (c, s_, g), synth.decode_x(seed, 1, K)))
-    step_bytes = sum(decode_bytes(1, K, N) for K, N, _, _ in qs)
+    qs = oracle_weights(row_frac)
 
     def step():
         for K, N, q, x in qs:
             oracle.linear_w4a16(x, *q)
 
+    gbs, dt, passes = _rate(step, sum(decode_bytes(1, K, N) for K, N, _, _ in qs) / 1e9, min_seconds)
+    return gbs, dt, passes, oracle.num_threads()
+
+
+def oracle_single_thread(seconds: float = 4.0, row_frac: int = 16):
+    """The headline sample on one host thread (a child process with
+    OMP_NUM_THREADS=1): {value, unit, cores, sample}."""
+    code = (f"import json, bench; g, dt, n, th = bench.oracle_decode_sample({seconds}, {row_frac}); "
+            "print(json.dumps([g, dt, n, th]))")
+    env = dict(os.environ, OMP_NUM_THREADS="1", CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True,
+                       timeout=300)
+    if r.returncode != 0:
+        return {"error": (r.stderr or r.stdout)[-300:]}
+    g, dt, n, th = json.loads(r.stdout.strip().splitlines()[-1])
+    return {"value": round(g, 3), "unit": "GB/s", "cores": th,
+            "sample": f"the four linears at M=1 over every {row_frac}th weight row, {n} passes in {dt:.1f} s"}
+
+
+def oracle_per_config(seconds: float = 2.0) -> dict:
+    """The oracle, as it stands, on a bounded sample of each workload the
+    parity suite covers (all host threads): {name: {value, unit, sample}}."""
+    import oracle
+    from oracle import moe as omoe
+    from oracle import stack as ostack
+    from bit_linear_moe_b200 import synth
+    out = {}
+
+    w, x = synth.single(0)
+    q = oracle.quantize(w)
+    g, dt, n = _rate(lambda: oracle.linear_w4a16(x, *q), decode_bytes(1, 2048, 2048) / 1e9, seconds)
+    out["single_linear_m1_k2048_n2048"] = {"value": round(g, 3), "unit": "GB/s",
+                                           "sample": f"the whole linear, {n} passes in {dt:.1f} s"}
+
+    qs = oracle_weights(16)
+    xs = [synth.decode_x(i + 1, 32, K) for i, (K, N, _, _) in enumerate(qs)]
+
+    def dec32():
+        for (K, N, qq, _), xx in zip(qs, xs):
+            oracle.linear_w4a16(xx, *qq)
+
+    g, dt, n = _rate(dec32, sum(decode_bytes(32, K, N) for K, N, _, _ in qs) / 1e9, seconds)
+    out["dense27b_decode_m32"] = {"value": round(g, 3), "unit": "GB/s",
+                                  "sample": f"M=32, every 16th weight row of the four linears, {n} passes in {dt:.1f} s"}
+
+    # prefill: 8 of the 2048 rows (quantized with the whole batch's gs) x all weight rows
+    pre = []
+    for K, N, qq, _ in oracle_weights(1):
+        seed = [sd for _, k_, n_, sd in SHAPES if k_ == K and n_ == N][0]
+        xa, _ = synth.prefill_x(seed, 2048, K)
+        xc, xsc, xg = oracle.quantize(xa)
+        rows = np.arange(0, 2048, 256)
+        pre.append((K, N, (np.ascontiguousarray(xc[rows]), np.ascontiguousarray(xsc[rows]), xg), qq))
+
+    def prefill():
+        for K, N, xq, qq in pre:
+            oracle.linear_w4a4(xq, qq)
+
+    g, dt, n = _rate(prefill, sum(2 * 8 * N * K for K, N, _, _ in pre) / 1e12, seconds)
+    out["prefill_w4a4_m2048"] = {"value": round(g, 5), "unit": "TFLOP/s",
+                                 "sample": f"8 of the 2048 rows x the four full weights, {n} passes in {dt:.1f} s"}
+
+    # MoE layer, T = 1: router, top-10, the chosen experts' gate/up, SwiGLU, down, combine
+    E, H, I, k = synth.MOE_E, synth.MOE_H, synth.MOE_I, synth.MOE_K
+    wr = synth.moe_router()
+    h = synth.moe_hidden(1)
+    idx, _ = omoe.topk(omoe.router_logits(h, wr), k)
+    chosen = [int(e) for e in idx[0]]
+    gq, dq = [], []
+    for e in chosen:
+        wgu, wd = synth.moe_expert(e)
+        gq.append(oracle.quantize(wgu))
+        dq.append(oracle.quantize(wd))
+    stk = lambda qq: (np.stack([a[0] for a in qq]), np.stack([a[1] for a in qq]),
+                      np.array([a[2] for a in qq], np.float32))
+    gu_w, dn_w = stk(gq), stk(dq)
+    local = {e: j for j, e in enumerate(chosen)}
+
+    def layer():
+        logits = omoe.router_logits(h, wr)
+        ix, wt = omoe.topk(logits, k)
+        il = np.vectorize(local.get)(ix).astype(np.int32)
+        offsets, perm_tok, perm_slot, row_of = omoe.permute(il, k)
+        gu, _ = omoe.grouped_linear_w4a16(h, offsets, perm_tok, *gu_w, gather=True)
+        a = ostack.bf16_round(omoe.swiglu(gu))
+        d, _ = omoe.grouped_linear_w4a16(a, offsets, perm_tok, *dn_w, gather=False)
+        omoe.combine(d, wt, row_of)
+
+    touched = k * (2 * I * H + H * I) * 9 // 16
+    g, dt, n = _rate(layer, touched / 1e9, seconds)
+    out["moe_layer_t1"] = {"value": round(g, 3), "unit": "GB/s of touched expert weights",
+                           "sample": f"one token, all {E} router rows, its {k} experts, {n} passes in {dt:.1f} s"}
+    out["threads"] = oracle.num_threads()
+    return out
+
+
+def run_reference(args):
+    """The oracle as the reference arm on the headline workload: each step is
+    the four linears at M = 1.  Full weights when the whole run fits in about
+    two minutes of host time; otherwise every n-th weight row, and the line's
+    config says so."""
+    import oracle
+    qs = oracle_weights(1)
+
+    def step(qq):
+        for K, N, q, x in qq:
+            oracle.linear_w4a16(x, *q)
+
+    t = time.perf_counter()
+    step(qs)
+    t1 = time.perf_counter() - t
+    row_frac = max(1, int(np.ceil(t1 * (args.steps + args.warmup) / 120.0)))
+    if row_frac > 1:
+        qs = oracle_weights(row_frac)
+    step_bytes = sum(decode_bytes(1, K, N) for K, N, _, _ in qs)
     for _ in range(args.warmup):
-        step()
+        step(qs)
     t = time.perf_counter()
     for _ in range(args.steps):
-        step()
+        step(qs)
     dt = time.perf_counter() - t
     gbs = step_bytes * args.steps / dt / 1e9
-    sample = "each step: the four linears at M=1 over every 64th weight row"
+    config = workload_config(args.gpus)
+    if row_frac > 1:
+        sample = f"each step: the four linears at M=1 over every {row_frac}th weight row"
+        config["sample"] = sample
+    else:
+        sample = "each step: the whole workload (the four linears at M=1, all weight rows)"
     line = {
         "impl": "reference", "metric": METRIC, "value": round(gbs, 3), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp64 accumulate (CPU oracle)",
         "data": "synthetic, same generator as the native arm",
-        "config": {"workload": WORKLOAD, "M": 1},
+        "config": config,
+        "timing": "host wall clock around the timed steps (CPU oracle)",
         "cpu_baseline": {"value": round(gbs, 3), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(gbs, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -923,7 +1073,9 @@ def main():
     if rank == 0 and world == 1 and not args.quick:
         gbs, dt, passes, threads = oracle_decode_sample(min_seconds=10.0)
         line["cpu_baseline"] = {"value": round(gbs, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
-                                "sample": f"the four linears at M=1, full weights, {passes} passes in {dt:.1f} s"}
+                                "sample": f"the four linears at M=1, full weights, {passes} passes in {dt:.1f} s",
+                                "single_thread": oracle_single_thread(),
+                                "per_config": oracle_per_config()}
     if rank == 0:
         print(json.dumps(line))
     if dist:

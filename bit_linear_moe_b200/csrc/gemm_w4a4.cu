@@ -135,6 +135,9 @@ __global__ void __launch_bounds__(w4a4::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+    // A programmatic dependent of the activation quantizer: the setup above
+    // overlaps its tail; nothing it writes is read before this point.
+    griddep_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -269,9 +272,16 @@ static int launch_typed(const CUtensorMap& ma, const CUtensorMap& mb, const Gemm
     std::call_once(once,
                    [&] { cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<NB>::kSmemBytes); });
     const int64_t ncols = (EPI == NVFP4_EPI_SWIGLU) ? a.N / 2 : a.N;
-    dim3 grid((unsigned)m_tiles, (unsigned)((ncols + BN - 1) / BN));
-    kern<<<grid, kThreads, Cfg<NB>::kSmemBytes, st>>>(ma, mb, a);
-    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+    cudaLaunchAttribute attr[1];
+    set_pdl_attr(attr[0]);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)m_tiles, (unsigned)((ncols + BN - 1) / BN));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = Cfg<NB>::kSmemBytes;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, ma, mb, a) == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 
 int launch_gemm_w4a4(const uint8_t* a_codes, const uint8_t* a_scales, const float* gs_a, int64_t M, int64_t K,

@@ -4,30 +4,35 @@
 // Pass 1 (amax_kernel) reduces max|x| over the tensor into one word of the
 // caller's workspace (non-negative floats order like their bit patterns, so an
 // unsigned atomicMax is exact and order-independent).  Pass 2
-// (quantize_kernel) gives one thread per 16-element block:
+// (quantize_kernel) gives one thread to each 16-element block:
 //     gs     = gs_in, or amax / 2688 (1 if amax == 0)     binary32, one rounding
 //     denom  = gs * 6
 //     s      = E4M3(amax_block / denom)                    nearest-even, satfinite
 //     r      = E4M3value(s) * gs
 //     code_i = E2M1(x_i / r), or +0 for the whole block when r == 0
-// The divisions are IEEE round-to-nearest (__fdiv_rn); nothing is contracted.
-// HBM-bound: pass 1 reads x once, pass 2 reads x again and writes 9/32 of its
-// bf16 size (codes + scales).
+// The quotients are those of IEEE round-to-nearest division; a reciprocal
+// product stands in for the division wherever it provably yields the same
+// code (e2m1x8_of_quotients).  Nothing is contracted.
+// HBM-bound: pass 1 reads x once, pass 2 reads x again (from L2 when x fits)
+// and writes 9/32 of its bf16 size (codes + scales).  Pass 2 is a
+// programmatic dependent of pass 1: its loads of x overlap pass 1's tail.
 #include "common.cuh"
 #include "internal.h"
+#include "tma.cuh"
 
 namespace nvfp4 {
 
+// Eight consecutive elements (16 bytes of bf16, 32 of fp32) -> fp32.
 template <typename T>
-struct Vec16;  // 16 consecutive elements -> fp32
+struct Vec8;
 
 template <>
-struct Vec16<__nv_bfloat16> {
-    static NVFP4_DEV void load(const __nv_bfloat16* p, float (&v)[16]) {
-        uint4 a = ldg_v4(p), b = ldg_v4(p + 8);
-        uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+struct Vec8<__nv_bfloat16> {
+    static NVFP4_DEV void load(const __nv_bfloat16* p, float (&v)[8]) {
+        const uint4 a = ldg_v4(p);
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
             v[2 * i] = bf16lo_to_f32(w[i]);
             v[2 * i + 1] = bf16hi_to_f32(w[i]);
         }
@@ -35,11 +40,11 @@ struct Vec16<__nv_bfloat16> {
 };
 
 template <>
-struct Vec16<float> {
-    static NVFP4_DEV void load(const float* p, float (&v)[16]) {
+struct Vec8<float> {
+    static NVFP4_DEV void load(const float* p, float (&v)[8]) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint4 a = ldg_v4(p + 4 * i);
+        for (int i = 0; i < 2; ++i) {
+            const uint4 a = ldg_v4(p + 4 * i);
             v[4 * i] = __uint_as_float(a.x);
             v[4 * i + 1] = __uint_as_float(a.y);
             v[4 * i + 2] = __uint_as_float(a.z);
@@ -48,19 +53,15 @@ struct Vec16<float> {
     }
 };
 
-template <typename T>
-__global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int64_t nvec16,
-                                                   unsigned* __restrict__ amax_bits) {
+NVFP4_DEV float amax8(const float (&v)[8]) {
     float m = 0.0f;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec16;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        float v[16];
-        Vec16<T>::load(x + i * 16, v);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(v[j]));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+    return m;
+}
+
+NVFP4_DEV void block_amax_to(float m, unsigned* amax_bits) {
+    m = warp_max(m);
     __shared__ float red[8];
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
     __syncthreads();
@@ -70,30 +71,45 @@ __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int6
     }
 }
 
-// max|x| over the rows src_rows[r] (r < nrows, entries < 0 skipped), 16 columns per item.
+// max|x| over n8 runs of eight elements, consecutive lanes on consecutive runs.
+template <typename T>
+__global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int64_t n8,
+                                                   unsigned* __restrict__ amax_bits) {
+    griddep_launch_dependents();  // the quantizer may start loading x now
+    float m = 0.0f;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    for (; i + 3 * stride < n8; i += 4 * stride) {  // four loads in flight per lane
+        float v[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) Vec8<T>::load(x + (i + u * stride) * 8, v[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) m = fmaxf(m, amax8(v[u]));
+    }
+    for (; i < n8; i += stride) {
+        float v[8];
+        Vec8<T>::load(x + i * 8, v);
+        m = fmaxf(m, amax8(v));
+    }
+    block_amax_to(m, amax_bits);
+}
+
+// max|x| over the rows src_rows[r] (r < nrows, entries < 0 skipped), eight columns per item.
 template <typename T>
 __global__ void __launch_bounds__(256) amax_rows_kernel(const T* __restrict__ x, const int32_t* __restrict__ src_rows,
                                                         int64_t nrows, int64_t cols, unsigned* __restrict__ amax_bits) {
+    griddep_launch_dependents();
     float m = 0.0f;
-    const int64_t nb = cols / 16, n = nrows * nb;
+    const int64_t nb = cols / 8, n = nrows * nb;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t r = i / nb, b = i % nb;
         const int32_t src = src_rows[r];
         if (src < 0) continue;
-        float v[16];
-        Vec16<T>::load(x + (int64_t)src * cols + b * 16, v);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(v[j]));
+        float v[8];
+        Vec8<T>::load(x + (int64_t)src * cols + b * 8, v);
+        m = fmaxf(m, amax8(v));
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    __shared__ float red[8];
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
-        atomicMax(amax_bits, __float_as_uint(m));
-    }
+    block_amax_to(m, amax_bits);
 }
 
 NVFP4_DEV float global_scale_from(const float* gs_in, const unsigned* amax_bits) {
@@ -102,61 +118,187 @@ NVFP4_DEV float global_scale_from(const float* gs_in, const unsigned* amax_bits)
     return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 2688.0f);
 }
 
-// One thread per (dst row, 16-element block) over the padded scale grid.
+// Approximate reciprocal (relative error below 2^-22 for normal inputs).
+NVFP4_DEV float rcp_approx(float a) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(a));
+    return r;
+}
+
+constexpr float kBracketLo = 0.99999618530273437500f;  // 1 - 2^-18
+constexpr float kBracketHi = 1.00000381469726562500f;  // 1 + 2^-18
+
+// E4M3 byte of RN(a / d), a >= 0 (the block scale).  inv ~ 1/d within 2^-22
+// (0 when d is 0, subnormal or not finite).  t = RN(a * inv) lies within
+// 2^-21 of RN(a / d); E4M3 rounding is monotone, so when t (1 - 2^-18) and
+// t (1 + 2^-18) give the same byte (one cvt converts both) it is the byte of
+// RN(a / d); otherwise the division decides.
+NVFP4_DEV uint32_t e4m3_of_quotient(float a, float d, float inv) {
+    if (inv != 0.0f) {
+        const float t = __fmul_rn(a, inv);
+        uint16_t pr;
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+            : "=h"(pr)
+            : "f"(__fmul_rn(t, kBracketHi)), "f"(__fmul_rn(t, kBracketLo)));
+        if ((pr & 0xFF) == (pr >> 8)) return pr & 0xFF;
+    }
+    return f32_to_e4m3(__fdiv_rn(a, d));
+}
+
+// E2M1 code (low nibble) of RN(v / r).
+NVFP4_DEV uint32_t e2m1_of_division(float v, float r) {
+    uint16_t pr;
+    asm("{\n\t.reg .b8 c;\n\tcvt.rn.satfinite.e2m1x2.f32 c, %1, %2;\n\tcvt.u16.u8 %0, c;\n\t}"
+        : "=h"(pr)
+        : "f"(0.0f), "f"(__fdiv_rn(v, r)));
+    return pr & 0xF;
+}
+
+// E2M1 codes of v[j] / r (j < 16, two words), each quotient the IEEE-rounded
+// division.  inv ~ 1/r within 2^-22 (0: always divide) and p = RN(v * inv)
+// put p within 2^-21 |v / r| of RN(v / r).  E2M1 rounding is monotone over
+// finite inputs (a NaN gives the same code either way), so where p (1 - 2^-18)
+// and p (1 + 2^-18) round to the same code, that is the code of RN(v / r); an
+// element whose bracket straddles a rounding boundary is divided.  (With bf16
+// inputs that is not rare: an element with the mantissa of the tensor's amax
+// makes v / r a boundary value in exact arithmetic, 0.75, 1.75 or 3.5, up to
+// the roundings of gs and r.)  A block whose amax / r is not below 15 (an
+// infinity, or near overflow) divides every element.
+NVFP4_DEV uint2 e2m1x16_of_quotients(const float (&v)[16], float amax, float r, float inv) {
+    uint32_t code[2], diff[2];
+    if (inv != 0.0f && __fmul_rn(amax, inv) < 15.0f) {
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            float lo[8], hi[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float p = __fmul_rn(v[8 * w + j], inv);
+                lo[j] = __fmul_rn(p, kBracketLo);
+                hi[j] = __fmul_rn(p, kBracketHi);
+            }
+            code[w] = f32x8_to_e2m1(hi);
+            diff[w] = f32x8_to_e2m1(lo) ^ code[w];
+        }
+    } else {
+        code[0] = code[1] = 0u;
+        diff[0] = diff[1] = 0xFFFFFFFFu;
+    }
+    if (diff[0] | diff[1]) {
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (diff[w] & (0xFu << (4 * j)))
+                    code[w] = (code[w] & ~(0xFu << (4 * j))) | (e2m1_of_division(v[8 * w + j], r) << (4 * j));
+    }
+    return make_uint2(code[0], code[1]);
+}
+
+// r is a normal float with a normal, finite reciprocal.
+NVFP4_DEV bool rcp_safe(float r) { return r >= 1.17549435e-38f && r <= 1.0e37f; }
+
+constexpr int kQThreads = 64;  // one CTA: 64 scale blocks (one per thread) of kQRows rows
+constexpr int kQRows = 2;      // rows per pass: their loads are issued together
+
+// Sixteen consecutive elements -> fp32 (two Vec8 loads).
+template <typename T>
+NVFP4_DEV void load16(const T* p, float (&v)[16]) {
+    float a[8], b[8];
+    Vec8<T>::load(p, a);
+    Vec8<T>::load(p + 8, b);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        v[j] = a[j];
+        v[8 + j] = b[j];
+    }
+}
+
+// CTA (blockIdx.x, row group g) quantizes the scale blocks b = 64 blockIdx.x +
+// t of rows 2 g', 2 g' + 1 for g' = blockIdx.y, blockIdx.y + gridDim.y, ...
+// (one thread per 16-element block; both rows' loads in flight before either
+// is used).  Grid: the padded scale grid (rows grid_rows, columns grid_cols).
 // src_rows (nullable): dst row r reads source row src_rows[r]; -1 marks a
 // padding row (zero codes and scales).  Rows >= dst_rows (tiled padding) and
 // scale columns >= cols/16 get zero scales and no codes.
+// row_bound (nullable): rows >= *row_bound are not touched at all.
 // row_inv (nullable): source row r is first normalised, x -> bf16(x * row_inv[r])
 // (the rows of nvfp4_rms_norm, recomputed instead of read back); x_ld is the
 // source row stride in elements.
+// Launched as a programmatic dependent of the pass that reduced amax_bits and
+// row_inv: x (complete before that pass began) is loaded first, the pass's
+// outputs only after griddep_wait().
 template <typename T, int LAYOUT>
-__global__ void __launch_bounds__(256) quantize_kernel(
+__global__ void __launch_bounds__(kQThreads) quantize_kernel(
     const T* __restrict__ x, const int32_t* __restrict__ src_rows, int64_t dst_rows, int64_t cols,
     int64_t grid_rows, int64_t grid_cols, const float* __restrict__ gs_in,
     const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ gs_out, const int32_t* __restrict__ row_bound, int64_t x_ld,
     const float* __restrict__ row_inv) {
-    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    const float gs = global_scale_from(gs_in, amax_bits);
-    if (i == 0 && gs_out) *gs_out = gs;
-    if (i >= grid_rows * grid_cols) return;
-    const int64_t r = i / grid_cols, b = i % grid_cols;
-    if (row_bound && r >= (int64_t)*row_bound) return;  // rows nobody reads (padded expert layout)
+    griddep_launch_dependents();
+    __shared__ float s_par[3];  // gs, denom, ~1/denom (0: divide)
+    const int t = threadIdx.x;
+    const int64_t b = (int64_t)blockIdx.x * kQThreads + t;
     const int64_t nsf = cols >> 4;
-    const int64_t soff = sf_offset<LAYOUT>(r, b, nsf);
-    int64_t src = r;
-    if (r < dst_rows && src_rows) src = src_rows[r];
-    if (r >= dst_rows || b >= nsf || src < 0) {
-        scales[soff] = 0;
-        if (r < dst_rows && b < nsf) *reinterpret_cast<uint2*>(codes + r * (cols >> 1) + b * 8) = make_uint2(0, 0);
-        return;
-    }
-    float v[16];
-    Vec16<T>::load(x + src * x_ld + b * 16, v);
-    if (row_inv) {
-        const float inv = row_inv[src];
+    const bool col_live = b < grid_cols, col_real = b < nsf;
+    const int64_t rbound = row_bound ? (int64_t)*row_bound : grid_rows;
+    const int64_t rend = rbound < grid_rows ? rbound : grid_rows;
+    const T* xb = x + b * 16;
+    uint8_t* cb = codes + b * 8;
+    bool waited = false;
+    for (int64_t r0 = (int64_t)blockIdx.y * kQRows; r0 < rend; r0 += (int64_t)gridDim.y * kQRows) {
+        float v[kQRows][16];
+        int64_t src[kQRows];
+        bool real[kQRows];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = __bfloat162float(__float2bfloat16_rn(v[j] * inv));
-    }
-    float amax_b = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) amax_b = fmaxf(amax_b, fabsf(v[j]));
-    const float denom = __fmul_rn(gs, 6.0f);
-    const uint32_t s = f32_to_e4m3(__fdiv_rn(amax_b, denom));
-    const float rsc = __fmul_rn(e4m3_to_f32(s), gs);
-    uint2 packed = make_uint2(0, 0);
-    if (rsc != 0.0f) {
-        float q0[8], q1[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            q0[j] = __fdiv_rn(v[j], rsc);
-            q1[j] = __fdiv_rn(v[8 + j], rsc);
+        for (int i = 0; i < kQRows; ++i) {
+            const int64_t r = r0 + i;
+            src[i] = r;
+            if (r < rend && r < dst_rows && src_rows) src[i] = src_rows[r];
+            real[i] = col_real && r < rend && r < dst_rows && src[i] >= 0;
+            if (real[i]) load16(xb + src[i] * x_ld, v[i]);
         }
-        packed.x = f32x8_to_e2m1(q0);
-        packed.y = f32x8_to_e2m1(q1);
+        if (!waited) {
+            griddep_wait();
+            if (t == 0) {
+                const float gs = global_scale_from(gs_in, amax_bits);
+                const float denom = __fmul_rn(gs, 6.0f);
+                s_par[0] = gs;
+                s_par[1] = denom;
+                s_par[2] = rcp_safe(denom) ? rcp_approx(denom) : 0.0f;
+                if (gs_out && blockIdx.x == 0 && blockIdx.y == 0) *gs_out = gs;
+            }
+            __syncthreads();
+            waited = true;
+        }
+        const float gs = s_par[0], denom = s_par[1], inv_denom = s_par[2];
+#pragma unroll
+        for (int i = 0; i < kQRows; ++i) {
+            const int64_t r = r0 + i;
+            if (!col_live || r >= rend) continue;
+            const int64_t soff = sf_offset<LAYOUT>(r, b, nsf);
+            uint2* cw = reinterpret_cast<uint2*>(cb + r * (cols >> 1));
+            if (!real[i]) {
+                scales[soff] = 0;
+                if (r < dst_rows && col_real) *cw = make_uint2(0u, 0u);
+                continue;
+            }
+            if (row_inv) {
+                const float inv = row_inv[src[i]];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[i][j] = __bfloat162float(__float2bfloat16_rn(v[i][j] * inv));
+            }
+            float amax_b = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) amax_b = fmaxf(amax_b, fabsf(v[i][j]));
+            const uint32_t sb = e4m3_of_quotient(amax_b, denom, inv_denom);
+            const float rsc = __fmul_rn(e4m3_to_f32(sb), gs);
+            uint2 packed = make_uint2(0u, 0u);
+            if (rsc != 0.0f)
+                packed = e2m1x16_of_quotients(v[i], amax_b, rsc, rcp_safe(rsc) ? rcp_approx(rsc) : 0.0f);
+            *cw = packed;
+            scales[soff] = (uint8_t)sb;
+        }
     }
-    *reinterpret_cast<uint2*>(codes + r * (cols >> 1) + b * 8) = packed;
-    scales[soff] = (uint8_t)s;
 }
 
 static int grid_for(int64_t n, int threads) {
@@ -166,21 +308,21 @@ static int grid_for(int64_t n, int threads) {
 
 int launch_amax(const void* x, int x_dtype, int64_t n, unsigned* amax_bits, cudaStream_t st) {
     if (cudaMemsetAsync(amax_bits, 0, sizeof(unsigned), st) != cudaSuccess) return NVFP4_ERR_LAUNCH;
-    const int64_t nvec = n / 16;
-    int grid = grid_for(nvec, 256);
+    const int64_t n8 = n / 8;
+    int grid = grid_for(n8, 256);
     const int cap = 148 * 8;
     if (grid > cap) grid = cap;
     if (x_dtype == NVFP4_DTYPE_BF16)
-        amax_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, nvec, amax_bits);
+        amax_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, n8, amax_bits);
     else
-        amax_kernel<float><<<grid, 256, 0, st>>>((const float*)x, nvec, amax_bits);
+        amax_kernel<float><<<grid, 256, 0, st>>>((const float*)x, n8, amax_bits);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 
 int launch_amax_rows(const void* x, const int32_t* src_rows, int64_t nrows, int64_t cols, unsigned* amax_bits,
                      cudaStream_t st) {
     if (cudaMemsetAsync(amax_bits, 0, sizeof(unsigned), st) != cudaSuccess) return NVFP4_ERR_LAUNCH;
-    int grid = grid_for(nrows * (cols / 16), 256);
+    int grid = grid_for(nrows * (cols / 8), 256);
     if (grid > 148 * 8) grid = 148 * 8;
     amax_rows_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, src_rows, nrows, cols, amax_bits);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
@@ -194,11 +336,25 @@ int launch_quantize(const void* x, int x_dtype, const int32_t* src_rows, int64_t
     const int64_t nsf = cols / 16;
     const int64_t grid_rows = sf_layout == NVFP4_SF_TILED ? (dst_rows + 127) / 128 * 128 : dst_rows;
     const int64_t grid_cols = sf_layout == NVFP4_SF_TILED ? (nsf + 3) / 4 * 4 : nsf;
-    const int grid = grid_for(grid_rows * grid_cols, 256);
-#define NVFP4_Q(T, L)                                                                                 \
-    quantize_kernel<T, L><<<grid, 256, 0, st>>>((const T*)x, src_rows, dst_rows, cols, grid_rows,     \
-                                                grid_cols, gs_in, amax_bits, codes, scales, gs_out, row_bound, \
-                                                x_ld, row_inv)
+    const int64_t gx = (grid_cols + kQThreads - 1) / kQThreads;
+    if (gx > 0x7fffffff) return NVFP4_ERR_SHAPE;
+    // With amax_bits from the pass just launched (no gs_in), a programmatic
+    // dependent of that pass; otherwise an ordinary launch.
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = {};
+    const int64_t gy = (grid_rows + kQRows - 1) / kQRows;
+    cfg.gridDim = dim3((unsigned)gx, (unsigned)(gy < 65535 ? gy : 65535));
+    cfg.blockDim = dim3(kQThreads);
+    cfg.stream = st;
+    if (!gs_in) {
+        set_pdl_attr(attr[0]);
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    cudaError_t e;
+#define NVFP4_Q(T, L)                                                                                         \
+    e = cudaLaunchKernelEx(&cfg, quantize_kernel<T, L>, (const T*)x, src_rows, dst_rows, cols, grid_rows,      \
+                           grid_cols, gs_in, amax_bits, codes, scales, gs_out, row_bound, x_ld, row_inv)
     if (x_dtype == NVFP4_DTYPE_BF16) {
         if (sf_layout == NVFP4_SF_TILED) NVFP4_Q(__nv_bfloat16, NVFP4_SF_TILED);
         else NVFP4_Q(__nv_bfloat16, NVFP4_SF_ROWMAJOR);
@@ -207,7 +363,7 @@ int launch_quantize(const void* x, int x_dtype, const int32_t* src_rows, int64_t
         else NVFP4_Q(float, NVFP4_SF_ROWMAJOR);
     }
 #undef NVFP4_Q
-    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
+    return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 
 }  // namespace nvfp4

@@ -90,3 +90,40 @@ def test_prefill_activations_with_outliers():
 def test_dense27b_weights_full(name, K, N, seed):
     w = synth.dense_weight(seed, K, N)
     _check(w, torch.float32, nv.SF_ROWMAJOR)
+
+
+def _e4m3_value(b):
+    """Value of an E4M3 byte (OCP FP8 format: bias 7, subnormals at exponent 0)."""
+    e, m = (b >> 3) & 15, b & 7
+    v = (1 + m / 8) * 2.0 ** (e - 7) if e else (m / 8) * 2.0 ** -6
+    return -v if b & 0x80 else v
+
+
+def test_quotients_at_e2m1_rounding_boundaries():
+    """Elements placed on, and a few fp32 ulps either side of, every E2M1
+    rounding boundary (the midpoints 0.25, 0.75, ..., 5 between E2M1 values)
+    of their block's scale r: the code must follow the IEEE-rounded quotient
+    x / r, ties to even, exactly as the oracle takes it."""
+    gs = np.float32(0.3712345)
+    mids = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
+    rng = np.random.default_rng(11)
+    rows = []
+    for _ in range(96):
+        x = np.zeros(16 * 16, np.float32)
+        for blk in range(16):
+            A = np.float32(rng.uniform(0.05, 40.0))
+            _, s, _ = oracle.quantize(np.concatenate([[A], np.zeros(15, np.float32)])[None, :].astype(np.float32),
+                                      gs=gs)
+            r = np.float32(np.float32(_e4m3_value(int(s[0, 0]))) * gs)
+            vals = [A]
+            for j in range(15):
+                v = np.float32(mids[j % 7] * np.float64(r))
+                for _ in range(abs(int(rng.integers(-3, 4)))):
+                    v = np.nextafter(v, np.float32(np.inf) if rng.random() < 0.5 else np.float32(0))
+                vals.append(-v if rng.random() < 0.5 else v)
+            x[16 * blk:16 * blk + 16] = vals
+        rows.append(x)
+    x = np.stack(rows)
+    _check(x, torch.float32, nv.SF_ROWMAJOR, gs_in=gs)
+    _check(x, torch.float32, nv.SF_TILED, gs_in=gs)
+    _check(x, torch.float32, nv.SF_TILED)  # the tensor's own gs: same boundaries, other scales
