@@ -603,7 +603,7 @@ int moe_grouped_linear(const void* x, int x_dtype, int64_t K, int gather, const 
         GroupedW4A4Ws w = grouped_w4a4_ws(ws, R, K, N, E, k, epilogue);
         NVFP4_TRY(launch_moe_pad(expert_offsets, E, rp, gather ? perm_tok : nullptr, w.pad_off, w.tile_info,
                                  w.src_rows, st));
-        NVFP4_TRY(launch_amax_rows(x, w.src_rows, rp, K, w.amax, st));
+        NVFP4_TRY(launch_amax_rows(x, w.src_rows, rp, K, w.amax, st, w.pad_off + E));
         NVFP4_TRY(launch_quantize(x, NVFP4_DTYPE_BF16, w.src_rows, rp, K, NVFP4_SF_TILED, nullptr, w.amax, w.codes,
                                   w.scales, w.gs_x, st, w.pad_off + E));
         const int64_t sf_stride = (int64_t)scales_bytes(N, K, NVFP4_SF_TILED);

@@ -35,9 +35,10 @@ int launch_quantize(const void* x, int x_dtype, const int32_t* src_rows, int64_t
                     int sf_layout, const float* gs_in, const unsigned* amax_bits, uint8_t* codes,
                     uint8_t* scales, float* gs_out, cudaStream_t st, const int32_t* row_bound = nullptr,
                     int64_t x_ld = 0, const float* row_inv = nullptr);
-// amax over bf16 rows x[src_rows[r]], r < nrows (negative entries skipped).
+// amax over bf16 rows x[src_rows[r]], r < nrows (negative entries skipped);
+// row_bound (nullable, device): rows >= *row_bound are not read.
 int launch_amax_rows(const void* x, const int32_t* src_rows, int64_t nrows, int64_t cols, unsigned* amax_bits,
-                     cudaStream_t st);
+                     cudaStream_t st, const int32_t* row_bound = nullptr);
 
 // gemv.cu: W4A16 on CUDA cores.
 struct GemvArgs {

@@ -94,20 +94,37 @@ __global__ void __launch_bounds__(256) amax_kernel(const T* __restrict__ x, int6
     block_amax_to(m, amax_bits);
 }
 
-// max|x| over the rows src_rows[r] (r < nrows, entries < 0 skipped), eight columns per item.
+// max|x| over the rows src_rows[r] (r < nrows, or < *row_bound when given;
+// entries < 0 skipped).  A CTA's 256 threads are 256 / tpr rows of tpr
+// 16-byte pieces (tpr = 2^lg_tpr, the largest power of two <= 256 dividing a
+// row's pieces), four such row groups in flight at once; CTAs take row groups
+// round-robin.
 template <typename T>
 __global__ void __launch_bounds__(256) amax_rows_kernel(const T* __restrict__ x, const int32_t* __restrict__ src_rows,
-                                                        int64_t nrows, int64_t cols, unsigned* __restrict__ amax_bits) {
+                                                        int64_t nrows, const int32_t* __restrict__ row_bound,
+                                                        int64_t cols, int lg_tpr, unsigned* __restrict__ amax_bits) {
     griddep_launch_dependents();
     float m = 0.0f;
-    const int64_t nb = cols / 8, n = nrows * nb;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / nb, b = i % nb;
-        const int32_t src = src_rows[r];
-        if (src < 0) continue;
-        float v[8];
-        Vec8<T>::load(x + (int64_t)src * cols + b * 8, v);
-        m = fmaxf(m, amax8(v));
+    const int64_t nb = cols / 8;
+    const int rpp = 256 >> lg_tpr;  // rows per pass
+    const int lr = threadIdx.x >> lg_tpr, c0 = threadIdx.x & ((1 << lg_tpr) - 1);
+    const int64_t rend = row_bound && (int64_t)*row_bound < nrows ? (int64_t)*row_bound : nrows;
+    for (int64_t r0 = (int64_t)blockIdx.x * 4 * rpp; r0 < rend; r0 += (int64_t)gridDim.x * 4 * rpp) {
+        int32_t src[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t r = r0 + u * rpp + lr;
+            src[u] = r < rend ? src_rows[r] : -1;
+        }
+        for (int64_t c = c0; c < nb; c += (1 << lg_tpr)) {
+            float v[4][8];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (src[u] >= 0) Vec8<T>::load(x + (int64_t)src[u] * cols + c * 8, v[u]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (src[u] >= 0) m = fmaxf(m, amax8(v[u]));
+        }
     }
     block_amax_to(m, amax_bits);
 }
@@ -197,8 +214,8 @@ NVFP4_DEV uint2 e2m1x16_of_quotients(const float (&v)[16], float amax, float r, 
 // r is a normal float with a normal, finite reciprocal.
 NVFP4_DEV bool rcp_safe(float r) { return r >= 1.17549435e-38f && r <= 1.0e37f; }
 
-constexpr int kQThreads = 64;  // one CTA: 64 scale blocks (one per thread) of kQRows rows
-constexpr int kQRows = 2;      // rows per pass: their loads are issued together
+constexpr int kQThreads = 128;  // one CTA: 128 threads, one 16-element block each
+constexpr int kQRows = 2;       // row passes per iteration: their loads are issued together
 
 // Sixteen consecutive elements -> fp32 (two Vec8 loads).
 template <typename T>
@@ -213,10 +230,14 @@ NVFP4_DEV void load16(const T* p, float (&v)[16]) {
     }
 }
 
-// CTA (blockIdx.x, row group g) quantizes the scale blocks b = 64 blockIdx.x +
-// t of rows 2 g', 2 g' + 1 for g' = blockIdx.y, blockIdx.y + gridDim.y, ...
-// (one thread per 16-element block; both rows' loads in flight before either
-// is used).  Grid: the padded scale grid (rows grid_rows, columns grid_cols).
+// One thread per (row, 16-element block) of the padded scale grid (rows
+// grid_rows, columns grid_cols).  A CTA's 128 threads are rpc = 128 / cw rows
+// of cw consecutive blocks (cw = 2^lg_cw, the largest power of two <= 128
+// dividing the padded column count, so short rows fill whole CTAs):
+// thread t takes block blockIdx.x * cw + (t mod cw) of row
+// r0 + i * rpc + t / cw, for i < 2 (both rows' loads in flight before either
+// is used) and r0 = 2 rpc (blockIdx.y + j gridDim.y); the grid is capped so
+// that each CTA walks several row groups.
 // src_rows (nullable): dst row r reads source row src_rows[r]; -1 marks a
 // padding row (zero codes and scales).  Rows >= dst_rows (tiled padding) and
 // scale columns >= cols/16 get zero scales and no codes.
@@ -233,11 +254,13 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(
     int64_t grid_rows, int64_t grid_cols, const float* __restrict__ gs_in,
     const unsigned* __restrict__ amax_bits, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ gs_out, const int32_t* __restrict__ row_bound, int64_t x_ld,
-    const float* __restrict__ row_inv) {
+    const float* __restrict__ row_inv, int lg_cw) {
     griddep_launch_dependents();
     __shared__ float s_par[3];  // gs, denom, ~1/denom (0: divide)
     const int t = threadIdx.x;
-    const int64_t b = (int64_t)blockIdx.x * kQThreads + t;
+    const int rpc = kQThreads >> lg_cw;
+    const int64_t b = ((int64_t)blockIdx.x << lg_cw) + (t & ((1 << lg_cw) - 1));
+    const int r_local = t >> lg_cw;
     const int64_t nsf = cols >> 4;
     const bool col_live = b < grid_cols, col_real = b < nsf;
     const int64_t rbound = row_bound ? (int64_t)*row_bound : grid_rows;
@@ -245,13 +268,13 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(
     const T* xb = x + b * 16;
     uint8_t* cb = codes + b * 8;
     bool waited = false;
-    for (int64_t r0 = (int64_t)blockIdx.y * kQRows; r0 < rend; r0 += (int64_t)gridDim.y * kQRows) {
+    for (int64_t r0 = (int64_t)blockIdx.y * rpc * kQRows; r0 < rend; r0 += (int64_t)gridDim.y * rpc * kQRows) {
         float v[kQRows][16];
         int64_t src[kQRows];
         bool real[kQRows];
 #pragma unroll
         for (int i = 0; i < kQRows; ++i) {
-            const int64_t r = r0 + i;
+            const int64_t r = r0 + i * rpc + r_local;
             src[i] = r;
             if (r < rend && r < dst_rows && src_rows) src[i] = src_rows[r];
             real[i] = col_real && r < rend && r < dst_rows && src[i] >= 0;
@@ -273,7 +296,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(
         const float gs = s_par[0], denom = s_par[1], inv_denom = s_par[2];
 #pragma unroll
         for (int i = 0; i < kQRows; ++i) {
-            const int64_t r = r0 + i;
+            const int64_t r = r0 + i * rpc + r_local;
             if (!col_live || r >= rend) continue;
             const int64_t soff = sf_offset<LAYOUT>(r, b, nsf);
             uint2* cw = reinterpret_cast<uint2*>(cb + r * (cols >> 1));
@@ -320,11 +343,16 @@ int launch_amax(const void* x, int x_dtype, int64_t n, unsigned* amax_bits, cuda
 }
 
 int launch_amax_rows(const void* x, const int32_t* src_rows, int64_t nrows, int64_t cols, unsigned* amax_bits,
-                     cudaStream_t st) {
+                     cudaStream_t st, const int32_t* row_bound) {
     if (cudaMemsetAsync(amax_bits, 0, sizeof(unsigned), st) != cudaSuccess) return NVFP4_ERR_LAUNCH;
-    int grid = grid_for(nrows * (cols / 8), 256);
+    const int64_t nb = cols / 8;
+    int lg_tpr = 0;  // the largest power of two <= 256 dividing a row's 16-byte pieces
+    while (lg_tpr < 8 && nb % (2 << lg_tpr) == 0) ++lg_tpr;
+    const int64_t rows_per_cta = (int64_t)(256 >> lg_tpr) * 4;
+    int grid = grid_for((nrows + rows_per_cta - 1) / rows_per_cta, 1);
     if (grid > 148 * 8) grid = 148 * 8;
-    amax_rows_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, src_rows, nrows, cols, amax_bits);
+    amax_rows_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>((const __nv_bfloat16*)x, src_rows, nrows, row_bound, cols,
+                                                          lg_tpr, amax_bits);
     return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_LAUNCH;
 }
 
@@ -336,14 +364,23 @@ int launch_quantize(const void* x, int x_dtype, const int32_t* src_rows, int64_t
     const int64_t nsf = cols / 16;
     const int64_t grid_rows = sf_layout == NVFP4_SF_TILED ? (dst_rows + 127) / 128 * 128 : dst_rows;
     const int64_t grid_cols = sf_layout == NVFP4_SF_TILED ? (nsf + 3) / 4 * 4 : nsf;
-    const int64_t gx = (grid_cols + kQThreads - 1) / kQThreads;
+    int lg_cw = 0;  // the largest power of two <= 128 dividing grid_cols
+    while (lg_cw < 7 && grid_cols % (2 << lg_cw) == 0) ++lg_cw;
+    const int64_t gx = grid_cols >> lg_cw;
     if (gx > 0x7fffffff) return NVFP4_ERR_SHAPE;
+    const int64_t rows_per_cta = (int64_t)(kQThreads >> lg_cw) * kQRows;
+    int64_t gy = (grid_rows + rows_per_cta - 1) / rows_per_cta;
+    // about one resident wave (8 CTAs of 128 threads per SM at 64 registers):
+    // each CTA walks several row groups
+    const int64_t gy_cap = (148 * 8 + gx - 1) / gx;
+    if (gy > gy_cap) gy = gy_cap;
+    if (gy > 65535) gy = 65535;
+    if (gy < 1) gy = 1;
     // With amax_bits from the pass just launched (no gs_in), a programmatic
     // dependent of that pass; otherwise an ordinary launch.
     cudaLaunchAttribute attr[1];
     cudaLaunchConfig_t cfg = {};
-    const int64_t gy = (grid_rows + kQRows - 1) / kQRows;
-    cfg.gridDim = dim3((unsigned)gx, (unsigned)(gy < 65535 ? gy : 65535));
+    cfg.gridDim = dim3((unsigned)gx, (unsigned)gy);
     cfg.blockDim = dim3(kQThreads);
     cfg.stream = st;
     if (!gs_in) {
@@ -354,7 +391,7 @@ int launch_quantize(const void* x, int x_dtype, const int32_t* src_rows, int64_t
     cudaError_t e;
 #define NVFP4_Q(T, L)                                                                                         \
     e = cudaLaunchKernelEx(&cfg, quantize_kernel<T, L>, (const T*)x, src_rows, dst_rows, cols, grid_rows,      \
-                           grid_cols, gs_in, amax_bits, codes, scales, gs_out, row_bound, x_ld, row_inv)
+                           grid_cols, gs_in, amax_bits, codes, scales, gs_out, row_bound, x_ld, row_inv, lg_cw)
     if (x_dtype == NVFP4_DTYPE_BF16) {
         if (sf_layout == NVFP4_SF_TILED) NVFP4_Q(__nv_bfloat16, NVFP4_SF_TILED);
         else NVFP4_Q(__nv_bfloat16, NVFP4_SF_ROWMAJOR);
