@@ -370,9 +370,11 @@ int launch_quantize(const void* x, int x_dtype, const int32_t* src_rows, int64_t
     if (gx > 0x7fffffff) return NVFP4_ERR_SHAPE;
     const int64_t rows_per_cta = (int64_t)(kQThreads >> lg_cw) * kQRows;
     int64_t gy = (grid_rows + rows_per_cta - 1) / rows_per_cta;
-    // about one resident wave (8 CTAs of 128 threads per SM at 64 registers):
-    // each CTA walks several row groups
-    const int64_t gy_cap = (148 * 8 + gx - 1) / gx;
+    // about four resident waves (8 CTAs of 128 threads per SM at 64
+    // registers): enough CTAs to hide the tail, few enough that each walks
+    // several row groups (measured: one wave left M = 8192 x 5120 at 64 us,
+    // four give 55 us; uncapped 64-thread CTAs, 59 us)
+    const int64_t gy_cap = (148 * 32 + gx - 1) / gx;
     if (gy > gy_cap) gy = gy_cap;
     if (gy > 65535) gy = 65535;
     if (gy < 1) gy = 1;
